@@ -1,0 +1,288 @@
+/*
+ * CPU oracle for the DeepSeek Sparse Attention (DSA) hot path.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the bench's
+ * CPU-baseline leg may load this library.  The GPU product path never calls it,
+ * and it shares no code, header, table or helper with the CUDA sources.
+ *
+ * Plain fp64 loops, one query row per call, written straight from the
+ * definitions on the pages:
+ *   - indexer score, "DeepSeek-V3.2" analysis page (PaperTrace), sec. 1.1, eq. (1)
+ *   - top-k selection set S_t, same page, sec. 1.1, eq. (2) and eq. (4)
+ *   - attention over the selected latents in MLA's MQA mode, same page,
+ *     sec. 1.1 eq. (2) and the MQA-mode paragraph (shared 576-d latent,
+ *     512 value dims); renormalised form, sec. 5.2 eq. (19)
+ *   - target distribution p: main-attention probabilities summed over heads
+ *     and L1-normalised, "DSA Continued Pre-Training" page, Stage 1
+ *   - sparse-stage indexer loss L^I = sum_t KL(p[t,S_t] || Softmax(I[t,S_t])),
+ *     "DSA Continued Pre-Training" page, Stage 2, and the analysis page eq. (4)
+ *
+ * Readings where the pages are silent (each also listed in the design notes):
+ *   - causal visibility includes the query's own position: s <= t;
+ *   - the indexer has no extra scale or dequantisation factors (eq. (1) as printed);
+ *   - masked scores (s > t) are -infinity;
+ *   - ties in top-k go to the smaller key index;
+ *   - value = latent dims [0, d_v), key = all d_qk latent dims;
+ *   - "main attention scores" are post-softmax probabilities;
+ *   - KL uses natural logs, 0 * ln 0 = 0, and is summed (not averaged) over t.
+ *
+ * Parity pins: every function here is pinned by a CPU test against a value or
+ * property fixed independently of this file (hand-worked example, library
+ * routines in fp64, closed forms, invariants).  None is "parity unpinned".
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#include <pthread.h>
+
+/* ---- storage decoders ------------------------------------------------------------------- */
+
+/* OCP FP8 E4M3 (fn variant): 1 sign, 4 exponent (bias 7), 3 mantissa bits; no infinities;
+ * exponent 15 with mantissa 7 is NaN; exponent 0 is subnormal m/8 * 2^-6. */
+double ref_e4m3_to_double(uint8_t b) {
+  int sign = (b >> 7) & 1;
+  int e = (b >> 3) & 0xF;
+  int m = b & 7;
+  double v;
+  if (e == 15 && m == 7) return NAN;
+  if (e == 0)
+    v = ldexp((double)m / 8.0, -6);
+  else
+    v = ldexp(1.0 + (double)m / 8.0, e - 7);
+  return sign ? -v : v;
+}
+
+/* bfloat16 = the top 16 bits of an IEEE binary32. */
+double ref_bf16_to_double(uint16_t h) {
+  uint32_t u = (uint32_t)h << 16;
+  float f;
+  memcpy(&f, &u, 4);
+  return (double)f;
+}
+
+/* ---- a1: lightning indexer, eq. (1) ----------------------------------------------------- */
+/* I[t,s] = sum_j w[t,j] * ReLU(q_I[t,j] . k_I[s]) for s <= t; -inf for s > t.
+ * q_row: [H_I][d_I] e4m3 of this query; k_seq: [Lk][d_I] e4m3 of its sequence;
+ * w_row: [H_I]; out: [Lk]. */
+void ref_indexer_row(const uint8_t* q_row, const uint8_t* k_seq, const float* w_row, int Lk,
+                     int t, int H_I, int d_I, double* out) {
+  for (int s = 0; s < Lk; ++s) {
+    if (s > t) {
+      out[s] = -INFINITY;
+      continue;
+    }
+    double score = 0.0;
+    for (int j = 0; j < H_I; ++j) {
+      double dot = 0.0;
+      for (int d = 0; d < d_I; ++d)
+        dot += ref_e4m3_to_double(q_row[j * d_I + d]) * ref_e4m3_to_double(k_seq[(int64_t)s * d_I + d]);
+      double relu = dot > 0.0 ? dot : 0.0;
+      score += (double)w_row[j] * relu;
+    }
+    out[s] = score;
+  }
+}
+
+/* ---- a2: top-k selection S_t, eq. (2)/(4) ----------------------------------------------- */
+typedef struct {
+  double score;
+  int32_t s;
+} scored_t;
+
+static int by_score_desc_then_index(const void* a, const void* b) {
+  const scored_t* x = (const scored_t*)a;
+  const scored_t* y = (const scored_t*)b;
+  if (x->score > y->score) return -1;
+  if (x->score < y->score) return 1;
+  return (x->s < y->s) ? -1 : (x->s > y->s);
+}
+
+/* S_t = the min(k, t+1) positions s <= t with the largest scores; ties -> smaller s.
+ * Full sort of all candidates, then the first entries.  idx[0..n) holds them in ascending
+ * position order, idx[n..k) = -1.  Returns n. */
+int ref_topk_row(const double* scores, int t, int k, int32_t* idx) {
+  int n_cand = t + 1;
+  scored_t* c = (scored_t*)malloc(sizeof(scored_t) * (size_t)n_cand);
+  for (int s = 0; s < n_cand; ++s) {
+    c[s].score = scores[s];
+    c[s].s = s;
+  }
+  qsort(c, (size_t)n_cand, sizeof(scored_t), by_score_desc_then_index);
+  int n = n_cand < k ? n_cand : k;
+  /* mark the chosen positions, then list them in ascending order */
+  unsigned char* chosen = (unsigned char*)calloc((size_t)n_cand, 1);
+  for (int i = 0; i < n; ++i) chosen[c[i].s] = 1;
+  int w = 0;
+  for (int s = 0; s < n_cand; ++s)
+    if (chosen[s]) idx[w++] = s;
+  for (int i = n; i < k; ++i) idx[i] = -1;
+  free(chosen);
+  free(c);
+  return n;
+}
+
+/* ---- a3/a4: attention in MQA mode over the selected latents ----------------------------- */
+/* For each head h: z_i = scale * <q[h,:], c[idx_i,:]> over all d_qk dims (valid i only),
+ * P_h,i = softmax_i(z), o[h,:] = sum_i P_h,i * c[idx_i, 0:d_v], lse[h] = ln sum_i exp(z_i).
+ * q_row: [H][d_qk] bf16; kv_seq: [Lk][d_qk] bf16; idx: [k] (-1 = empty slot).
+ * out: [H][d_v]; lse: [H] (nullable); P: [H][k] (nullable, 0 for empty slots). */
+void ref_sparse_mla_row(const uint16_t* q_row, const uint16_t* kv_seq, const int32_t* idx, int k,
+                        int H, int d_qk, int d_v, double scale, double* out, double* lse,
+                        double* P) {
+  double* z = (double*)malloc(sizeof(double) * (size_t)(k > 0 ? k : 1));
+  for (int h = 0; h < H; ++h) {
+    double m = -INFINITY;
+    for (int i = 0; i < k; ++i) {
+      if (idx[i] < 0) continue;
+      double dot = 0.0;
+      for (int d = 0; d < d_qk; ++d)
+        dot += ref_bf16_to_double(q_row[h * d_qk + d]) *
+               ref_bf16_to_double(kv_seq[(int64_t)idx[i] * d_qk + d]);
+      z[i] = scale * dot;
+      if (z[i] > m) m = z[i];
+    }
+    double denom = 0.0;
+    for (int i = 0; i < k; ++i)
+      if (idx[i] >= 0) denom += exp(z[i] - m);
+    for (int e = 0; e < d_v; ++e) out[h * d_v + e] = 0.0;
+    for (int i = 0; i < k; ++i) {
+      double p = idx[i] >= 0 ? exp(z[i] - m) / denom : 0.0;
+      if (P) P[(int64_t)h * k + i] = p;
+      if (idx[i] < 0) continue;
+      for (int e = 0; e < d_v; ++e)
+        out[h * d_v + e] += p * ref_bf16_to_double(kv_seq[(int64_t)idx[i] * d_qk + e]);
+    }
+    if (lse) lse[h] = m + log(denom);
+  }
+  free(z);
+}
+
+/* Target distribution over S_t ("DSA Continued Pre-Training", Stage 1 and Stage 2):
+ * main-attention probabilities summed over all heads, then L1-normalised along the
+ * selected positions.  P: [H][k] from ref_sparse_mla_row.  p: [k], 0 for empty slots. */
+void ref_p_sel_row(const double* P, const int32_t* idx, int k, int H, double* p) {
+  double total = 0.0;
+  for (int i = 0; i < k; ++i) {
+    double acc = 0.0;
+    if (idx[i] >= 0)
+      for (int h = 0; h < H; ++h) acc += P[(int64_t)h * k + i];
+    p[i] = acc;
+    total += acc;
+  }
+  for (int i = 0; i < k; ++i) p[i] = total > 0.0 ? p[i] / total : 0.0;
+}
+
+/* ---- a5: sparse-stage indexer loss, one row of eq. (4) ---------------------------------- */
+/* KL(p || q) with q = Softmax(I[t, S_t]) over the valid selected positions:
+ * sum_i p_i (ln p_i - ln q_i), ln q_i = I_i - ln sum_j exp(I_j); terms with p_i = 0 are 0. */
+double ref_kl_row(const double* scores_row, const int32_t* idx, const double* p, int k) {
+  double m = -INFINITY;
+  for (int i = 0; i < k; ++i)
+    if (idx[i] >= 0 && scores_row[idx[i]] > m) m = scores_row[idx[i]];
+  double denom = 0.0;
+  for (int i = 0; i < k; ++i)
+    if (idx[i] >= 0) denom += exp(scores_row[idx[i]] - m);
+  double log_z = m + log(denom);
+  double kl = 0.0;
+  for (int i = 0; i < k; ++i) {
+    if (idx[i] < 0 || p[i] == 0.0) continue;
+    double log_q = scores_row[idx[i]] - log_z;
+    kl += p[i] * (log(p[i]) - log_q);
+  }
+  return kl;
+}
+
+/* ---- dense causal MQA over all s <= t (for the k >= t+1 and eq. (19)/(20) checks) ------- */
+void ref_dense_mla_row(const uint16_t* q_row, const uint16_t* kv_seq, int t, int H, int d_qk,
+                       int d_v, double scale, double* out, double* lse, double* A /* [H][t+1] */) {
+  int n = t + 1;
+  int32_t* all = (int32_t*)malloc(sizeof(int32_t) * (size_t)n);
+  for (int s = 0; s < n; ++s) all[s] = s;
+  ref_sparse_mla_row(q_row, kv_seq, all, n, H, d_qk, d_v, scale, out, lse, A);
+  free(all);
+}
+
+/* ---- whole-path driver over a set of query rows (CPU baseline timing) ------------------- */
+/* Runs indexer -> top-k -> sparse MLA (-> p -> KL when emit_p) for each listed flat row
+ * r = b*Lq + i, rows spread over nthreads POSIX threads; each row is computed by the
+ * single-threaded functions above, so threading changes no arithmetic.
+ * Outputs per listed row j: scores [Lk], idx [k], out [H][d_v], lse [H], p [k], kl [1].
+ * Any output pointer may be NULL. */
+typedef struct {
+  const uint8_t *qI, *kI;
+  const float* w;
+  const uint16_t *q, *kv;
+  const int64_t* rows;
+  int64_t nrows;
+  int B, Lq, Lk, H_I, d_I, k, H, d_qk, d_v, emit_p;
+  double scale;
+  double *scores, *out, *lse, *p, *kl;
+  int32_t* idx;
+  int tid, nthreads;
+  /* which inputs are stored densely per listed row rather than for every row */
+  int rows_packed;
+} path_job_t;
+
+static void* path_worker(void* arg) {
+  path_job_t* J = (path_job_t*)arg;
+  double* sc = (double*)malloc(sizeof(double) * (size_t)J->Lk);
+  int32_t* id = (int32_t*)malloc(sizeof(int32_t) * (size_t)J->k);
+  double* o = (double*)malloc(sizeof(double) * (size_t)J->H * J->d_v);
+  double* l = (double*)malloc(sizeof(double) * (size_t)J->H);
+  double* P = (double*)malloc(sizeof(double) * (size_t)J->H * J->k);
+  double* pp = (double*)malloc(sizeof(double) * (size_t)J->k);
+  for (int64_t j = J->tid; j < J->nrows; j += J->nthreads) {
+    int64_t r = J->rows[j];
+    int b = (int)(r / J->Lq), i = (int)(r % J->Lq);
+    int t = i + J->Lk - J->Lq;
+    int64_t src = J->rows_packed ? j : r;
+    const uint8_t* q_row = J->qI + src * J->H_I * J->d_I;
+    const uint8_t* k_seq = J->kI + (int64_t)b * J->Lk * J->d_I;
+    const float* w_row = J->w + src * J->H_I;
+    ref_indexer_row(q_row, k_seq, w_row, J->Lk, t, J->H_I, J->d_I, sc);
+    ref_topk_row(sc, t, J->k, id);
+    const uint16_t* qa = J->q + src * J->H * J->d_qk;
+    const uint16_t* kvs = J->kv + (int64_t)b * J->Lk * J->d_qk;
+    ref_sparse_mla_row(qa, kvs, id, J->k, J->H, J->d_qk, J->d_v, J->scale, o, l,
+                       J->emit_p ? P : NULL);
+    double klv = 0.0;
+    if (J->emit_p) {
+      ref_p_sel_row(P, id, J->k, J->H, pp);
+      klv = ref_kl_row(sc, id, pp, J->k);
+    }
+    if (J->scores) memcpy(J->scores + j * J->Lk, sc, sizeof(double) * (size_t)J->Lk);
+    if (J->idx) memcpy(J->idx + j * J->k, id, sizeof(int32_t) * (size_t)J->k);
+    if (J->out) memcpy(J->out + j * J->H * J->d_v, o, sizeof(double) * (size_t)J->H * J->d_v);
+    if (J->lse) memcpy(J->lse + j * J->H, l, sizeof(double) * (size_t)J->H);
+    if (J->p && J->emit_p) memcpy(J->p + j * J->k, pp, sizeof(double) * (size_t)J->k);
+    if (J->kl) J->kl[j] = klv;
+  }
+  free(sc);
+  free(id);
+  free(o);
+  free(l);
+  free(P);
+  free(pp);
+  return NULL;
+}
+
+int ref_path_rows(const uint8_t* qI, const uint8_t* kI, const float* w, const uint16_t* q,
+                  const uint16_t* kv, int rows_packed, const int64_t* rows, int64_t nrows, int B,
+                  int Lq, int Lk, int H_I, int d_I, int k, int H, int d_qk, int d_v, double scale,
+                  int emit_p, double* scores, int32_t* idx, double* out, double* lse, double* p,
+                  double* kl, int nthreads) {
+  if (nthreads < 1) nthreads = 1;
+  pthread_t* th = (pthread_t*)malloc(sizeof(pthread_t) * (size_t)nthreads);
+  path_job_t* jobs = (path_job_t*)malloc(sizeof(path_job_t) * (size_t)nthreads);
+  for (int i = 0; i < nthreads; ++i) {
+    path_job_t J = {qI, kI, w, q, kv, rows, nrows, B, Lq, Lk, H_I, d_I, k, H, d_qk, d_v, emit_p,
+                    scale, scores, out, lse, p, kl, idx, i, nthreads, rows_packed};
+    jobs[i] = J;
+    pthread_create(&th[i], NULL, path_worker, &jobs[i]);
+  }
+  for (int i = 0; i < nthreads; ++i) pthread_join(th[i], NULL);
+  free(th);
+  free(jobs);
+  return 0;
+}
