@@ -62,6 +62,7 @@ def _load():
         lib.dsa_gen_uniform_int.argtypes = [u64, u64, i64, i64, i32, i32, vp]
         lib.dsa_gen_normal_f64.argtypes = [u64, u64, i64, i64, vp]
         lib.dsa_gen_normal_bf16.argtypes = [u64, u64, i64, i64, vp]
+        lib.dsa_gen_e4m3_small_int.argtypes = [u64, u64, i64, i64, vp]
         _lib = lib
     return _lib
 
@@ -90,6 +91,13 @@ def normal_bf16_bits(seed: int, tensor_id: int, n: int, offset: int = 0) -> np.n
     assert offset % 2 == 0
     out = np.empty(n, dtype=np.uint16)
     _load().dsa_gen_normal_bf16(seed, tensor_id, offset, n, out.ctypes.data)
+    return out
+
+
+def e4m3_small_int(seed: int, tensor_id: int, n: int, offset: int = 0) -> np.ndarray:
+    """The [-3, 3] integer stream (same draws as uniform_int(..., -3, 3)) as e4m3 bytes."""
+    out = np.empty(n, dtype=np.uint8)
+    _load().dsa_gen_e4m3_small_int(seed, tensor_id, offset, n, out.ctypes.data)
     return out
 
 
@@ -159,18 +167,16 @@ def q_index(wl: Workload, row0: int = 0, nrows: int | None = None) -> np.ndarray
     """q_I rows [row0, row0+nrows) of [B*Lq, H_I, d_I], e4m3 bytes."""
     nrows = wl.rows - row0 if nrows is None else nrows
     per = wl.H_I * wl.d_I
-    v = uniform_int(wl.seed, TENSOR_Q_I, nrows * per, -3, 3, offset=row0 * per)
-    return int_to_e4m3(v).reshape(nrows, wl.H_I, wl.d_I)
+    return e4m3_small_int(wl.seed, TENSOR_Q_I, nrows * per, offset=row0 * per).reshape(
+        nrows, wl.H_I, wl.d_I)
 
 
 def k_index(wl: Workload, b: int | None = None) -> np.ndarray:
     """k_I of sequence b ([Lk, d_I]) or of all sequences ([B, Lk, d_I]), e4m3 bytes."""
     per = wl.Lk * wl.d_I
     if b is None:
-        v = uniform_int(wl.seed, TENSOR_K_I, wl.B * per, -3, 3)
-        return int_to_e4m3(v).reshape(wl.B, wl.Lk, wl.d_I)
-    v = uniform_int(wl.seed, TENSOR_K_I, per, -3, 3, offset=b * per)
-    return int_to_e4m3(v).reshape(wl.Lk, wl.d_I)
+        return e4m3_small_int(wl.seed, TENSOR_K_I, wl.B * per).reshape(wl.B, wl.Lk, wl.d_I)
+    return e4m3_small_int(wl.seed, TENSOR_K_I, per, offset=b * per).reshape(wl.Lk, wl.d_I)
 
 
 def w_index(wl: Workload, row0: int = 0, nrows: int | None = None) -> np.ndarray:

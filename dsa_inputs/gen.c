@@ -94,3 +94,16 @@ void dsa_gen_normal_bf16(uint64_t seed, uint64_t tensor_id, int64_t offset, int6
     if (2 * j + 1 < n) out[2 * j + 1] = f32_to_bf16_rne((float)b);
   }
 }
+
+/* Integers uniform in [-3, 3] (the int stream with lo=-3, hi=3) stored as OCP e4m3fn bytes:
+ * -3 0xC4, -2 0xC0, -1 0xB8, 0 0x00, 1 0x38, 2 0x40, 3 0x44 (exact encodings). */
+void dsa_gen_e4m3_small_int(uint64_t seed, uint64_t tensor_id, int64_t offset, int64_t n,
+                            uint8_t* out) {
+  static const uint8_t enc[7] = {0xC4, 0xC0, 0xB8, 0x00, 0x38, 0x40, 0x44};
+  const uint64_t key = stream_key(seed, tensor_id);
+#pragma omp parallel for schedule(static)
+  for (int64_t i = 0; i < n; ++i) {
+    uint64_t x = word_at(key, (uint64_t)(offset + i)) >> 32;
+    out[i] = enc[(x * 7u) >> 32];
+  }
+}

@@ -1,0 +1,150 @@
+/*
+ * dsa.h - C ABI of the DeepSeek Sparse Attention (DSA) hot path on NVIDIA B200 (sm_100a).
+ *
+ * The path, as defined by the DeepSeek-V3.2 pages:
+ *   1. lightning-indexer scores      ("DeepSeek-V3.2" analysis page, sec. 1.1, eq. (1))
+ *   2. per-query top-k selection S_t (same page, sec. 1.1, eq. (2) and the S_t of eq. (4))
+ *   3. attention in MLA's MQA mode over only the selected latent entries c_s
+ *      (same page, sec. 1.1, eq. (2) and the MQA-mode paragraph; V3.2-Exp page, sec. 1)
+ *   4. the sparse-stage indexer loss L^I = sum_t KL(p[t,S_t] || Softmax(I[t,S_t]))
+ *      ("DSA Continued Pre-Training" page, Stage 2; analysis page eq. (4)), where p is the
+ *      main attention summed over heads and L1-normalised ("DSA Continued Pre-Training",
+ *      Stage 1).
+ *
+ * Shapes and positions.  B sequences; Lq queries and Lk keys per sequence.  Query i of a
+ * sequence sits at absolute position t = i + (Lk - Lq) and sees keys s <= t (prefill:
+ * Lq == Lk; decode: Lq == 1 and the query sees its whole context).
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller, dense, row-major,
+ *     contiguous, 16-byte aligned.  The library never allocates, frees or synchronises
+ *     (except dsa_last_device_status, which is documented as synchronising).
+ *   - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL = legacy default).
+ *   - Arguments are validated on the host before any launch; a failed check returns
+ *     DSA_ERR_INVALID_ARG (bad pointer, size or alignment) or DSA_ERR_UNSUPPORTED (a shape
+ *     outside the compiled kernels) and launches nothing.
+ *   - A launch failure returns DSA_ERR_CUDA.  The device must be sm_100 (B200) or the call
+ *     returns DSA_ERR_NO_SM100.
+ *   - Every wait inside a kernel is bounded in time; on expiry the kernel records
+ *     DSA_ERR_TIMEOUT in a device status word and exits.  dsa_last_device_status reads it.
+ *   - `ws` / `ws_bytes` is caller-owned device scratch of at least dsa_workspace_bytes()
+ *     for the same op and sizes (ws may be NULL when that size is 0).
+ */
+#ifndef DSA_H_
+#define DSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  DSA_OK = 0,
+  DSA_ERR_INVALID_ARG = 1,
+  DSA_ERR_UNSUPPORTED = 2,
+  DSA_ERR_CUDA = 3,
+  DSA_ERR_NO_SM100 = 4,
+  DSA_ERR_TIMEOUT = 5
+} dsa_status;
+
+/* A cudaStream_t passed through the ABI without CUDA headers. */
+typedef void* dsa_stream_t;
+
+enum { DSA_OP_INDEXER = 0, DSA_OP_TOPK = 1, DSA_OP_SPARSE_MLA_FWD = 2, DSA_OP_INDEXER_KL = 3 };
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* dsa_status_str(dsa_status s);
+
+/* ABI version of this library (major*100 + minor). */
+int dsa_version(void);
+
+/* Bytes of scratch the op needs for these sizes on the CURRENT device (0 if none).
+ * op: DSA_OP_*.  Unused size arguments are ignored (pass 0).  Returns 0 for unknown ops. */
+size_t dsa_workspace_bytes(int op, int B, int Lq, int Lk, int k, int H);
+
+/*
+ * Lightning indexer ("DeepSeek-V3.2" analysis page, sec. 1.1, eq. (1)):
+ *   scores[b,i,s] = sum_{j<H_I} w[b,i,j] * max(0, sum_{d<d_I} q_I[b,i,j,d] * k_I[b,s,d])
+ * for s <= t(i), and -infinity for s > t(i).
+ *   q_fp8  [B, Lq, H_I, d_I]  FP8 E4M3 (OCP "fn"), one byte per element
+ *   k_fp8  [B, Lk, d_I]       FP8 E4M3, the single shared key head
+ *   w      [B, Lq, H_I]       fp32 per-head weights
+ *   scores [B, Lq, Lk]        fp32 output
+ * Products are exact in FP8 and accumulate in fp32 on the tensor cores; the ReLU, the
+ * w-weighted head sum and the causal mask run in fp32 in the epilogue, so the
+ * [Lq, Lk, H_I] intermediate is never written.  For integer-valued inputs whose
+ * partial sums stay below 2^24 ulps the result is exact (bit-identical to fp64).
+ * Supported: (H_I, d_I) with H_I in {4, 8, 16, 32, 64} and d_I in {32, 64, 128};
+ * 1 <= Lq <= Lk.  ws: unused (pass NULL, 0).
+ */
+dsa_status dsa_indexer(const void* q_fp8, const void* k_fp8, const float* w, float* scores, int B,
+                       int Lq, int Lk, int H_I, int d_I, void* ws, size_t ws_bytes,
+                       dsa_stream_t stream);
+
+/*
+ * Top-k selection ("DeepSeek-V3.2" analysis page, sec. 1.1, eq. (2); S_t of eq. (4)):
+ * for each query row, the n = min(k, t+1) positions s <= t with the largest scores.
+ * Ties are broken toward the smaller position, so the set is unique.
+ *   scores [B, Lq, Lk] fp32 (only s <= t is read)
+ *   idx    [B, Lq, k]  int32 output: the n selected positions in ascending order,
+ *                      then -1 in slots n..k-1
+ * Scores must not be NaN.  Supported: 1 <= k <= 4096, Lk <= 262144.
+ * ws: unused (pass NULL, 0).
+ */
+dsa_status dsa_topk(const float* scores, int32_t* idx, int B, int Lq, int Lk, int k, void* ws,
+                    size_t ws_bytes, dsa_stream_t stream);
+
+/*
+ * Sparse attention in MLA's MQA mode over the selected latents ("DeepSeek-V3.2" analysis
+ * page, sec. 1.1, eq. (2) and the MQA-mode paragraph; renormalised form eq. (19)).
+ * Every query head shares the latent entry c_s = kv[b,s,:]; keys use all d_qk dims,
+ * values are dims [0, d_v).  For each head h of query (b,i), over the valid slots
+ * (idx >= 0) of idx[b,i,:]:
+ *   z_h,j = scale * <q[b,i,h,:], kv[b,idx_j,:]>,   P_h,j = softmax_j(z_h,:)
+ *   out[b,i,h,:] = sum_j P_h,j * kv[b,idx_j,0:d_v],  lse[b,i,h] = ln sum_j exp(z_h,j)
+ * If p_sel is not NULL it also writes the head-summed, L1-normalised target
+ * ("DSA Continued Pre-Training" page, Stage 1/2):
+ *   p_sel[b,i,j] = sum_h P_h,j / sum_j' sum_h P_h,j'   (= sum_h P_h,j / H), 0 for empty slots.
+ *   q_bf16  [B, Lq, H, d_qk] bf16     kv_bf16 [B, Lk, d_qk] bf16    idx [B, Lq, k] int32
+ *   out_bf16 [B, Lq, H, d_v] bf16     lse [B, Lq, H] fp32 (nullable)
+ *   p_sel   [B, Lq, k] fp32 (nullable)
+ * Every valid idx must lie in [0, Lk); each row needs at least one valid slot.
+ * bf16 tensor-core products with fp32 accumulation and fp32 softmax; bf16 output (RNE).
+ * Supported: H <= 128, (d_qk, d_v) in {(576, 512), (80, 64)}, 1 <= k <= 65536.
+ * ws: dsa_workspace_bytes(DSA_OP_SPARSE_MLA_FWD, B, Lq, Lk, k, H) bytes (split-KV partials
+ * when there are too few query rows to fill the GPU; 0 otherwise).
+ */
+dsa_status dsa_sparse_mla_fwd(const void* q_bf16, const void* kv_bf16, const int32_t* idx, int B,
+                              int Lq, int Lk, int H, int d_qk, int d_v, int k, float scale,
+                              void* out_bf16, float* lse, float* p_sel, void* ws, size_t ws_bytes,
+                              dsa_stream_t stream);
+
+/*
+ * Sparse-stage indexer loss ("DSA Continued Pre-Training" page, Stage 2; "DeepSeek-V3.2"
+ * analysis page, eq. (4)):
+ *   L^I = sum_{b,i} sum_{j valid} p[b,i,j] * (ln p[b,i,j] - ln q[b,i,j]),
+ *   q[b,i,:] = Softmax over the valid slots of scores[b,i,idx[b,i,:]],  0 * ln 0 = 0.
+ *   scores [B, Lq, Lk] fp32, idx [B, Lq, k] int32, p_sel [B, Lq, k] fp32
+ *   loss   device pointer to one fp32 (written)
+ *   loss_per_query [B, Lq] fp32 (nullable): the per-row KL terms
+ * fp32 per-row arithmetic; the sum over rows is taken in a fixed order (deterministic).
+ * ws: dsa_workspace_bytes(DSA_OP_INDEXER_KL, B, Lq, 0, k, 0) bytes.
+ */
+dsa_status dsa_indexer_kl(const float* scores, const int32_t* idx, const float* p_sel, int B,
+                          int Lq, int Lk, int k, float* loss, float* loss_per_query, void* ws,
+                          size_t ws_bytes, dsa_stream_t stream);
+
+/*
+ * Waits for `stream`, then returns and clears the device status word that kernels set
+ * when a bounded wait expires (DSA_ERR_TIMEOUT) - DSA_OK if none did.  Synchronising;
+ * meant for tests and diagnostics.  Returns DSA_ERR_CUDA if the stream itself failed.
+ */
+dsa_status dsa_last_device_status(dsa_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_H_ */

@@ -1,0 +1,182 @@
+"""Python binding of libdsa.so, the DSA hot path on B200 (sm_100a).
+
+Argument marshalling only: every function checks the torch tensors it is given
+(device, dtype, shape, contiguity), passes their device pointers and the current
+CUDA stream to the C entry point of the same name, and raises DsaError on a
+non-zero status.  All arithmetic runs in the library's CUDA kernels; there is no
+CPU path.  Layouts and semantics are those of include/dsa.h.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+from . import build as _build
+
+__all__ = [
+    "DsaError", "load", "dsa_status_str", "dsa_version", "dsa_workspace_bytes", "dsa_indexer",
+    "dsa_topk", "dsa_sparse_mla_fwd", "dsa_indexer_kl", "dsa_last_device_status",
+    "DSA_OP_INDEXER", "DSA_OP_TOPK", "DSA_OP_SPARSE_MLA_FWD", "DSA_OP_INDEXER_KL", "EXPORTED",
+]
+
+DSA_OP_INDEXER, DSA_OP_TOPK, DSA_OP_SPARSE_MLA_FWD, DSA_OP_INDEXER_KL = 0, 1, 2, 3
+EXPORTED = ("dsa_status_str", "dsa_version", "dsa_workspace_bytes", "dsa_indexer", "dsa_topk",
+            "dsa_sparse_mla_fwd", "dsa_indexer_kl", "dsa_last_device_status")
+
+
+class DsaError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn} failed: {dsa_status_str(code)} ({code})")
+        self.code = code
+
+
+_lib = None
+
+
+def load(rebuild: bool = False) -> ctypes.CDLL:
+    """Load (building first if missing or stale) the in-tree libdsa.so."""
+    global _lib
+    if _lib is None or rebuild:
+        path = _build.LIB
+        if rebuild or _build.stale():
+            path = _build.build()
+        lib = ctypes.CDLL(path)
+        vp, i32, sz, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_float
+        lib.dsa_status_str.argtypes = [i32]
+        lib.dsa_status_str.restype = ctypes.c_char_p
+        lib.dsa_version.restype = i32
+        lib.dsa_workspace_bytes.argtypes = [i32, i32, i32, i32, i32, i32]
+        lib.dsa_workspace_bytes.restype = sz
+        lib.dsa_indexer.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, vp, sz, vp]
+        lib.dsa_topk.argtypes = [vp, vp, i32, i32, i32, i32, vp, sz, vp]
+        lib.dsa_sparse_mla_fwd.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, f32, vp,
+                                           vp, vp, vp, sz, vp]
+        lib.dsa_indexer_kl.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, vp, vp, sz, vp]
+        lib.dsa_last_device_status.argtypes = [vp]
+        for name in ("dsa_indexer", "dsa_topk", "dsa_sparse_mla_fwd", "dsa_indexer_kl",
+                     "dsa_last_device_status"):
+            getattr(lib, name).restype = i32
+        _lib = lib
+    return _lib
+
+
+def dsa_status_str(code: int) -> str:
+    return load().dsa_status_str(int(code)).decode()
+
+
+def dsa_version() -> int:
+    return load().dsa_version()
+
+
+def dsa_workspace_bytes(op: int, B: int, Lq: int, Lk: int, k: int, H: int) -> int:
+    return int(load().dsa_workspace_bytes(op, B, Lq, Lk, k, H))
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(t: torch.Tensor, name: str, dtype, shape) -> None:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _raise(fn: str, code: int) -> None:
+    if code != 0:
+        raise DsaError(fn, code)
+
+
+def _ws(ws):
+    if ws is None:
+        return None, 0
+    if ws.device.type != "cuda" or not ws.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    return ctypes.c_void_p(ws.data_ptr()), ws.numel() * ws.element_size()
+
+
+def dsa_indexer(q_fp8: torch.Tensor, k_fp8: torch.Tensor, w: torch.Tensor, scores: torch.Tensor,
+                stream=None) -> None:
+    """scores[B,Lq,Lk] = lightning-indexer scores (eq. (1)) of q_I [B,Lq,H_I,d_I] e4m3,
+    k_I [B,Lk,d_I] e4m3 and w [B,Lq,H_I] fp32; -inf above the causal diagonal."""
+    B, Lq, H_I, d_I = q_fp8.shape
+    Lk = k_fp8.shape[1]
+    _check(q_fp8, "q_fp8", torch.float8_e4m3fn, (B, Lq, H_I, d_I))
+    _check(k_fp8, "k_fp8", torch.float8_e4m3fn, (B, Lk, d_I))
+    _check(w, "w", torch.float32, (B, Lq, H_I))
+    _check(scores, "scores", torch.float32, (B, Lq, Lk))
+    _raise("dsa_indexer", load().dsa_indexer(_ptr(q_fp8), _ptr(k_fp8), _ptr(w), _ptr(scores), B, Lq,
+                                             Lk, H_I, d_I, None, 0, _stream(stream)))
+
+
+def dsa_topk(scores: torch.Tensor, idx: torch.Tensor, stream=None) -> None:
+    """idx[B,Lq,k] = ascending positions of the top-k scores of each row (s <= t), ties to the
+    smaller position, -1 padded."""
+    B, Lq, Lk = scores.shape
+    k = idx.shape[2]
+    _check(scores, "scores", torch.float32, (B, Lq, Lk))
+    _check(idx, "idx", torch.int32, (B, Lq, k))
+    _raise("dsa_topk", load().dsa_topk(_ptr(scores), _ptr(idx), B, Lq, Lk, k, None, 0,
+                                       _stream(stream)))
+
+
+def dsa_sparse_mla_fwd(q: torch.Tensor, kv: torch.Tensor, idx: torch.Tensor, scale: float,
+                       out: torch.Tensor, lse: torch.Tensor | None = None,
+                       p_sel: torch.Tensor | None = None, ws: torch.Tensor | None = None,
+                       stream=None) -> None:
+    """MQA-mode attention of q [B,Lq,H,d_qk] over the selected latents kv[b, idx] (bf16);
+    out [B,Lq,H,d_v] bf16, optional lse [B,Lq,H] and head-summed p_sel [B,Lq,k] (fp32)."""
+    B, Lq, H, d_qk = q.shape
+    Lk = kv.shape[1]
+    k = idx.shape[2]
+    d_v = out.shape[3]
+    _check(q, "q", torch.bfloat16, (B, Lq, H, d_qk))
+    _check(kv, "kv", torch.bfloat16, (B, Lk, d_qk))
+    _check(idx, "idx", torch.int32, (B, Lq, k))
+    _check(out, "out", torch.bfloat16, (B, Lq, H, d_v))
+    if lse is not None:
+        _check(lse, "lse", torch.float32, (B, Lq, H))
+    if p_sel is not None:
+        _check(p_sel, "p_sel", torch.float32, (B, Lq, k))
+    wsp, wsb = _ws(ws)
+    _raise("dsa_sparse_mla_fwd",
+           load().dsa_sparse_mla_fwd(_ptr(q), _ptr(kv), _ptr(idx), B, Lq, Lk, H, d_qk, d_v, k,
+                                     float(scale), _ptr(out), _ptr(lse), _ptr(p_sel), wsp, wsb,
+                                     _stream(stream)))
+
+
+def dsa_indexer_kl(scores: torch.Tensor, idx: torch.Tensor, p_sel: torch.Tensor, loss: torch.Tensor,
+                   loss_per_query: torch.Tensor | None = None, ws: torch.Tensor | None = None,
+                   stream=None) -> None:
+    """loss[0] = sum over rows of KL(p_sel || Softmax(scores[idx])) (eq. (4))."""
+    B, Lq, Lk = scores.shape
+    k = idx.shape[2]
+    _check(scores, "scores", torch.float32, (B, Lq, Lk))
+    _check(idx, "idx", torch.int32, (B, Lq, k))
+    _check(p_sel, "p_sel", torch.float32, (B, Lq, k))
+    _check(loss, "loss", torch.float32, (1,))
+    if loss_per_query is not None:
+        _check(loss_per_query, "loss_per_query", torch.float32, (B, Lq))
+    wsp, wsb = _ws(ws)
+    _raise("dsa_indexer_kl",
+           load().dsa_indexer_kl(_ptr(scores), _ptr(idx), _ptr(p_sel), B, Lq, Lk, k, _ptr(loss),
+                                 _ptr(loss_per_query), wsp, wsb, _stream(stream)))
+
+
+def dsa_last_device_status(stream=None) -> int:
+    """Synchronise `stream` and return (and clear) the kernels' device status code."""
+    return int(load().dsa_last_device_status(_stream(stream)))

@@ -1,0 +1,400 @@
+// Host side of the C ABI declared in include/dsa.h: argument validation, launch-shape
+// selection, TMA descriptor encoding and kernel launches.  All kernels of the library are
+// compiled in this one translation unit so they share the device status word.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/dsa.h"
+#include "indexer.cuh"
+#include "indexer_kl.cuh"
+#include "ptx.cuh"
+#include "sparse_mla.cuh"
+#include "status.cuh"
+#include "topk.cuh"
+
+namespace {
+
+using dsa::g_device_status;
+
+// ------------------------------------------------------------------------------ device info
+struct DeviceInfo {
+  bool ok = false;
+  bool sm100 = false;
+  int sms = 0;
+};
+
+constexpr int kMaxDevices = 64;
+DeviceInfo g_dev[kMaxDevices];
+std::once_flag g_dev_once[kMaxDevices];
+
+dsa_status current_device(DeviceInfo& out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DSA_ERR_CUDA;
+  std::call_once(g_dev_once[dev], [dev]() {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return;
+    if (cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) return;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return;
+    g_dev[dev].sm100 = (major == 10 && minor == 0);
+    g_dev[dev].sms = sms;
+    g_dev[dev].ok = true;
+  });
+  if (!g_dev[dev].ok) return DSA_ERR_CUDA;
+  if (!g_dev[dev].sm100) return DSA_ERR_NO_SM100;
+  out = g_dev[dev];
+  return DSA_OK;
+}
+
+int sm_count_or_default() {
+  DeviceInfo d;
+  if (current_device(d) == DSA_OK) return d.sms;
+  return 148;
+}
+
+// ------------------------------------------------------------------------------ TMA encode
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, []() {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D row-major tensor [outer, inner] with `row_bytes` between rows; box [box_outer, box_inner].
+bool encode_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner,
+               uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+               CUtensorMapSwizzle swz) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline dsa_status launch_result() {
+  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------------------ indexer
+template <int H_I, int D_I, int G>
+dsa_status launch_indexer(const void* q, const void* kk, const float* w, float* scores, int B,
+                          int Lq, int Lk, int sms, cudaStream_t stream) {
+  using Cfg = dsa::indexer::Cfg<H_I, D_I, G>;
+  const CUtensorMapSwizzle swz = D_I == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                 : D_I == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                             : CU_TENSOR_MAP_SWIZZLE_32B;
+  CUtensorMap tm_q, tm_k;
+  if (!encode_2d(&tm_q, CU_TENSOR_MAP_DATA_TYPE_UINT8, q, D_I, static_cast<uint64_t>(B) * Lq * H_I,
+                 D_I, D_I, Cfg::N, swz))
+    return DSA_ERR_CUDA;
+  if (!encode_2d(&tm_k, CU_TENSOR_MAP_DATA_TYPE_UINT8, kk, D_I, static_cast<uint64_t>(B) * Lk, D_I,
+                 D_I, dsa::indexer::kTileKeys, swz))
+    return DSA_ERR_CUDA;
+  dsa::indexer::Params p{};
+  p.w = w;
+  p.scores = scores;
+  p.B = B;
+  p.Lq = Lq;
+  p.Lk = Lk;
+  p.n_qg = (Lq + G - 1) / G;
+  p.n_kt = (Lk + dsa::indexer::kTileKeys - 1) / dsa::indexer::kTileKeys;
+  const long base = static_cast<long>(B) * p.n_qg;
+  if (base >= 2L * sms) {
+    p.kc = p.n_kt;
+  } else {
+    const long splits = (4L * sms + base - 1) / base;
+    p.kc = static_cast<int>(std::max<long>(4, (p.n_kt + splits - 1) / splits));
+  }
+  p.kc = std::min(p.kc, p.n_kt);
+  p.n_kc = (p.n_kt + p.kc - 1) / p.kc;
+  const long items = base * p.n_kc;
+  if (items > INT32_MAX) return DSA_ERR_UNSUPPORTED;
+  p.n_items = static_cast<int>(items);
+  auto kern = dsa::indexer::indexer_kernel<H_I, D_I, G>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) !=
+      cudaSuccess)
+    return DSA_ERR_CUDA;
+  const int grid = static_cast<int>(std::min<long>(items, sms));
+  kern<<<grid, dsa::indexer::kThreads, Cfg::kSmemBytes, stream>>>(tm_q, tm_k, p);
+  return launch_result();
+}
+
+// ------------------------------------------------------------------------------ top-k
+template <int C>
+dsa_status launch_topk(const float* scores, int32_t* idx, int B, int Lq, int Lk, int k,
+                       cudaStream_t stream) {
+  const int slice = (Lk + C - 1) / C;
+  const size_t smem = static_cast<size_t>(slice) * sizeof(uint32_t);
+  auto kern = dsa::topk::topk_kernel<C>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(B) * Lq * C);
+  cfg.blockDim = dim3(dsa::topk::kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (C > 1 && cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 0) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  if (cudaLaunchKernelEx(&cfg, kern, scores, idx, B, Lq, Lk, k) != cudaSuccess) return DSA_ERR_CUDA;
+  return launch_result();
+}
+
+int topk_cluster_size(int rows, int Lk, int sms) {
+  int c = 1;
+  while (c < 8 && (Lk + c - 1) / c > dsa::topk::kMaxSlice) c *= 2;
+  while (c < 8 && static_cast<long>(rows) * c < sms && (Lk + 2 * c - 1) / (2 * c) >= 4096) c *= 2;
+  return c;
+}
+
+// ------------------------------------------------------------------------------ sparse MLA
+struct MlaSplit {
+  int n_split;
+  int per_split;
+};
+
+MlaSplit mla_split(int rows, int k, int n_dv, int sms, bool want_p) {
+  MlaSplit s{1, ((k + dsa::mla::kBN - 1) / dsa::mla::kBN) * dsa::mla::kBN};
+  const long ctas = static_cast<long>(rows) * n_dv;
+  if (want_p || ctas >= sms) return s;
+  int n = static_cast<int>(sms / ctas);
+  const int max_by_len = std::max(1, (k + 4 * dsa::mla::kBN - 1) / (4 * dsa::mla::kBN));
+  n = std::max(1, std::min(n, max_by_len));
+  const int blocks = (k + dsa::mla::kBN - 1) / dsa::mla::kBN;
+  s.per_split = ((blocks + n - 1) / n) * dsa::mla::kBN;
+  s.n_split = (k + s.per_split - 1) / s.per_split;
+  return s;
+}
+
+size_t mla_ws_bytes(int rows, int k, int H, int d_v, int sms) {
+  const int n_dv = d_v > 256 ? d_v / 256 : 1;
+  const MlaSplit s = mla_split(rows, k, n_dv, sms, false);
+  if (s.n_split <= 1) return 0;
+  return static_cast<size_t>(s.n_split) * rows * H * (static_cast<size_t>(d_v) + 1) * sizeof(float);
+}
+
+template <int D_QK, int D_V>
+dsa_status launch_mla(const void* q, const void* kv, const int32_t* idx, int B, int Lq, int Lk,
+                      int H, int k, float scale, void* out, float* lse, float* p_sel, void* ws,
+                      size_t ws_bytes, int sms, cudaStream_t stream) {
+  using Cfg = dsa::mla::Cfg<D_QK, D_V>;
+  const int rows = B * Lq;
+  const MlaSplit sp = mla_split(rows, k, Cfg::kNdv, sms, p_sel != nullptr);
+  dsa::mla::Params p{};
+  p.kv = static_cast<const __nv_bfloat16*>(kv);
+  p.idx = idx;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.p_sel = p_sel;
+  p.B = B;
+  p.Lq = Lq;
+  p.Lk = Lk;
+  p.H = H;
+  p.k = k;
+  p.n_split = sp.n_split;
+  p.per_split = sp.per_split;
+  p.scale_log2 = scale * dsa::mla::kLog2e;
+  if (sp.n_split > 1) {
+    const size_t need = static_cast<size_t>(sp.n_split) * rows * H * (static_cast<size_t>(D_V) + 1) * sizeof(float);
+    if (ws == nullptr || ws_bytes < need || !aligned16(ws)) return DSA_ERR_INVALID_ARG;
+    p.part_o = static_cast<float*>(ws);
+    p.part_lse = p.part_o + static_cast<size_t>(sp.n_split) * rows * H * D_V;
+  }
+  CUtensorMap tm_q;
+  if (!encode_2d(&tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, D_QK, static_cast<uint64_t>(rows) * H,
+                 static_cast<uint64_t>(D_QK) * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+    return DSA_ERR_CUDA;
+  auto kern = dsa::mla::sparse_mla_kernel<D_QK, D_V>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) !=
+      cudaSuccess)
+    return DSA_ERR_CUDA;
+  const long grid = static_cast<long>(rows) * Cfg::kNdv * sp.n_split;
+  if (grid > INT32_MAX) return DSA_ERR_UNSUPPORTED;
+  kern<<<static_cast<unsigned>(grid), dsa::mla::kThreads, Cfg::kSmemBytes, stream>>>(tm_q, p);
+  if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
+  if (sp.n_split > 1) {
+    dsa::mla::combine_kernel<D_V><<<rows * H, 128, 0, stream>>>(
+        p.part_o, p.part_lse, sp.n_split, rows * H, static_cast<__nv_bfloat16*>(out), lse);
+    return launch_result();
+  }
+  return DSA_OK;
+}
+
+}  // namespace
+
+// ================================================================================ C ABI
+extern "C" {
+
+const char* dsa_status_str(dsa_status s) {
+  switch (s) {
+    case DSA_OK: return "DSA_OK";
+    case DSA_ERR_INVALID_ARG: return "DSA_ERR_INVALID_ARG";
+    case DSA_ERR_UNSUPPORTED: return "DSA_ERR_UNSUPPORTED";
+    case DSA_ERR_CUDA: return "DSA_ERR_CUDA";
+    case DSA_ERR_NO_SM100: return "DSA_ERR_NO_SM100";
+    case DSA_ERR_TIMEOUT: return "DSA_ERR_TIMEOUT";
+  }
+  return "DSA_ERR_UNKNOWN";
+}
+
+int dsa_version(void) { return 100; }
+
+size_t dsa_workspace_bytes(int op, int B, int Lq, int Lk, int k, int H) {
+  (void)Lk;
+  if (B <= 0 || Lq <= 0) return 0;
+  const long rows = static_cast<long>(B) * Lq;
+  switch (op) {
+    case DSA_OP_SPARSE_MLA_FWD: {
+      if (k <= 0 || H <= 0) return 0;
+      const int sms = sm_count_or_default();
+      // an upper bound over every supported value width
+      return std::max(mla_ws_bytes(static_cast<int>(rows), k, H, 512, sms),
+                      mla_ws_bytes(static_cast<int>(rows), k, H, 64, sms));
+    }
+    case DSA_OP_INDEXER_KL:
+      return static_cast<size_t>(rows) * sizeof(float);
+    default:
+      return 0;
+  }
+}
+
+dsa_status dsa_indexer(const void* q_fp8, const void* k_fp8, const float* w, float* scores, int B,
+                       int Lq, int Lk, int H_I, int d_I, void* ws, size_t ws_bytes,
+                       dsa_stream_t stream) {
+  (void)ws;
+  (void)ws_bytes;
+  if (!q_fp8 || !k_fp8 || !w || !scores) return DSA_ERR_INVALID_ARG;
+  if (B <= 0 || Lq <= 0 || Lk <= 0 || Lq > Lk || H_I <= 0 || d_I <= 0) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q_fp8) || !aligned16(k_fp8) || !aligned16(w) || !aligned16(scores))
+    return DSA_ERR_INVALID_ARG;
+  if (static_cast<long>(B) * Lk > INT32_MAX || static_cast<long>(B) * Lq * H_I > INT32_MAX)
+    return DSA_ERR_UNSUPPORTED;
+  DeviceInfo dev;
+  const dsa_status ds = current_device(dev);
+  if (ds != DSA_OK) return ds;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const bool decode = (Lq == 1);
+  if (H_I == 64 && d_I == 128)
+    return decode ? launch_indexer<64, 128, 1>(q_fp8, k_fp8, w, scores, B, Lq, Lk, dev.sms, st)
+                  : launch_indexer<64, 128, 4>(q_fp8, k_fp8, w, scores, B, Lq, Lk, dev.sms, st);
+  if (H_I == 32 && d_I == 128)
+    return decode ? launch_indexer<32, 128, 1>(q_fp8, k_fp8, w, scores, B, Lq, Lk, dev.sms, st)
+                  : launch_indexer<32, 128, 8>(q_fp8, k_fp8, w, scores, B, Lq, Lk, dev.sms, st);
+  if (H_I == 16 && d_I == 128)
+    return launch_indexer<16, 128, 16>(q_fp8, k_fp8, w, scores, B, Lq, Lk, dev.sms, st);
+  if (H_I == 8 && d_I == 64)
+    return launch_indexer<8, 64, 32>(q_fp8, k_fp8, w, scores, B, Lq, Lk, dev.sms, st);
+  if (H_I == 4 && d_I == 32)
+    return launch_indexer<4, 32, 64>(q_fp8, k_fp8, w, scores, B, Lq, Lk, dev.sms, st);
+  return DSA_ERR_UNSUPPORTED;
+}
+
+dsa_status dsa_topk(const float* scores, int32_t* idx, int B, int Lq, int Lk, int k, void* ws,
+                    size_t ws_bytes, dsa_stream_t stream) {
+  (void)ws;
+  (void)ws_bytes;
+  if (!scores || !idx) return DSA_ERR_INVALID_ARG;
+  if (B <= 0 || Lq <= 0 || Lk <= 0 || Lq > Lk || k <= 0) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(scores) || !aligned16(idx)) return DSA_ERR_INVALID_ARG;
+  if (k > 4096 || Lk > 8 * dsa::topk::kMaxSlice) return DSA_ERR_UNSUPPORTED;
+  if (static_cast<long>(B) * Lq * 8 > INT32_MAX) return DSA_ERR_UNSUPPORTED;
+  DeviceInfo dev;
+  const dsa_status ds = current_device(dev);
+  if (ds != DSA_OK) return ds;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  switch (topk_cluster_size(B * Lq, Lk, dev.sms)) {
+    case 1: return launch_topk<1>(scores, idx, B, Lq, Lk, k, st);
+    case 2: return launch_topk<2>(scores, idx, B, Lq, Lk, k, st);
+    case 4: return launch_topk<4>(scores, idx, B, Lq, Lk, k, st);
+    default: return launch_topk<8>(scores, idx, B, Lq, Lk, k, st);
+  }
+}
+
+dsa_status dsa_sparse_mla_fwd(const void* q_bf16, const void* kv_bf16, const int32_t* idx, int B,
+                              int Lq, int Lk, int H, int d_qk, int d_v, int k, float scale,
+                              void* out_bf16, float* lse, float* p_sel, void* ws, size_t ws_bytes,
+                              dsa_stream_t stream) {
+  if (!q_bf16 || !kv_bf16 || !idx || !out_bf16) return DSA_ERR_INVALID_ARG;
+  if (B <= 0 || Lq <= 0 || Lk <= 0 || Lq > Lk || H <= 0 || k <= 0) return DSA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q_bf16) || !aligned16(kv_bf16) || !aligned16(idx) || !aligned16(out_bf16) ||
+      (lse && !aligned16(lse)) || (p_sel && !aligned16(p_sel)))
+    return DSA_ERR_INVALID_ARG;
+  if (H > 128 || k > 65536) return DSA_ERR_UNSUPPORTED;
+  if (static_cast<long>(B) * Lq * H * 2 * 8 > INT32_MAX) return DSA_ERR_UNSUPPORTED;
+  DeviceInfo dev;
+  const dsa_status ds = current_device(dev);
+  if (ds != DSA_OK) return ds;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (d_qk == 576 && d_v == 512)
+    return launch_mla<576, 512>(q_bf16, kv_bf16, idx, B, Lq, Lk, H, k, scale, out_bf16, lse, p_sel,
+                                ws, ws_bytes, dev.sms, st);
+  if (d_qk == 80 && d_v == 64)
+    return launch_mla<80, 64>(q_bf16, kv_bf16, idx, B, Lq, Lk, H, k, scale, out_bf16, lse, p_sel,
+                              ws, ws_bytes, dev.sms, st);
+  return DSA_ERR_UNSUPPORTED;
+}
+
+dsa_status dsa_indexer_kl(const float* scores, const int32_t* idx, const float* p_sel, int B,
+                          int Lq, int Lk, int k, float* loss, float* loss_per_query, void* ws,
+                          size_t ws_bytes, dsa_stream_t stream) {
+  if (!scores || !idx || !p_sel || !loss) return DSA_ERR_INVALID_ARG;
+  if (B <= 0 || Lq <= 0 || Lk <= 0 || Lq > Lk || k <= 0) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(scores) || !aligned16(idx) || !aligned16(p_sel) || (reinterpret_cast<uintptr_t>(loss) & 3u))
+    return DSA_ERR_INVALID_ARG;
+  const long rows = static_cast<long>(B) * Lq;
+  if (rows > INT32_MAX) return DSA_ERR_UNSUPPORTED;
+  float* per_row = loss_per_query;
+  if (per_row == nullptr) {
+    if (ws == nullptr || ws_bytes < static_cast<size_t>(rows) * sizeof(float)) return DSA_ERR_INVALID_ARG;
+    per_row = static_cast<float*>(ws);
+  }
+  DeviceInfo dev;
+  const dsa_status ds = current_device(dev);
+  if (ds != DSA_OK) return ds;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  dsa::kl::kl_rows_kernel<<<static_cast<unsigned>(rows), dsa::kl::kRowThreads, 0, st>>>(
+      scores, idx, p_sel, Lk, k, per_row);
+  if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
+  dsa::kl::kl_sum_kernel<<<1, dsa::kl::kSumThreads, 0, st>>>(per_row, static_cast<int>(rows), loss);
+  return launch_result();
+}
+
+dsa_status dsa_last_device_status(dsa_stream_t stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return DSA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(int)) != cudaSuccess) return DSA_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int)) != cudaSuccess) return DSA_ERR_CUDA;
+  return static_cast<dsa_status>(v & 0xFF);
+}
+
+}  // extern "C"

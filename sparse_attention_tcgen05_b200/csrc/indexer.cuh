@@ -1,0 +1,301 @@
+// Lightning indexer ("DeepSeek-V3.2" analysis page, sec. 1.1, eq. (1)) on sm_100a:
+//   I[t,s] = sum_j w[t,j] * ReLU(q_I[t,j] . k_I[s])   (s <= t),   -inf for s > t.
+//
+// One FP8 tcgen05 GEMM per tile: keys along M (128 TMEM lanes), (query, head) pairs along N
+// (G queries x H_I heads), K = d_I.  A thread of the epilogue owns one key row of the fp32
+// accumulator, so the ReLU, the w-weighted head sum and the causal mask are applied in
+// registers without any cross-lane reduction; only the [Lq, Lk] scores reach HBM.
+//
+// Persistent, warp-specialised CTA (one per SM):
+//   warp 0        TMA producer: the q_I group once per work item, then k_I tiles (6 stages)
+//   warp 1        MMA issuer (one thread): d_I/32 MMAs of 128 x N x 32 per tile
+//   warp 2        TMEM allocator (2 accumulators of N columns, double-buffered)
+//   warps 4..11   epilogue: tcgen05.ld -> ReLU * w -> head sum -> mask -> store
+// Work item = (sequence, group of G queries, chunk of key tiles); key tiles beyond the
+// group's last visible position skip the MMA and are written as -inf directly.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "ptx.cuh"
+
+namespace dsa {
+namespace indexer {
+
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 128 + kEpiWarps * 32;
+constexpr int kStages = 6;
+constexpr int kTileKeys = 128;
+
+struct Params {
+  const float* w;
+  float* scores;
+  int B, Lq, Lk;
+  int n_qg;   // query groups per sequence
+  int n_kt;   // key tiles per sequence
+  int kc;     // key tiles per work chunk
+  int n_kc;   // chunks per query group
+  int n_items;
+};
+
+template <int H_I, int D_I, int G>
+struct Cfg {
+  static constexpr int N = G * H_I;                      // MMA N (columns per accumulator)
+  static constexpr int kQBytes = N * D_I;                // q_I group tile
+  static constexpr int kKBytes = kTileKeys * D_I;        // k_I tile
+  static constexpr int kTmemCols = (2 * N <= 32) ? 32 : (2 * N <= 64) ? 64 : (2 * N <= 128) ? 128
+                                   : (2 * N <= 256) ? 256 : 512;
+  static constexpr bool kSplitWG = (G >= 2);             // two epilogue warpgroups split queries
+  static constexpr int kColsPerWG = kSplitWG ? N / 2 : N;
+  static constexpr int kQPerWG = kSplitWG ? G / 2 : 1;
+  static constexpr int kEpiWorkers = kSplitWG ? 256 : 128;
+  static constexpr uint32_t kSwizzle = D_I == 128 ? kSw128 : D_I == 64 ? kSw64 : kSw32;
+  static constexpr uint32_t kIdesc = make_idesc(0, 0, false, false, 128, N);
+  // shared memory layout (offsets from a 1024-aligned base)
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffK = kOffQ + 2 * ((kQBytes + 1023) / 1024) * 1024;
+  static constexpr int kOffW = kOffK + kStages * kKBytes;
+  static constexpr int kOffBar = kOffW + 2 * N * 4;
+  static constexpr int kNumBars = 2 * kStages + 8;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
+  static_assert(N % 16 == 0 && N >= 16 && N <= 256, "MMA N");
+  static_assert(kColsPerWG % 32 == 0, "epilogue column split");
+  static_assert(D_I % 32 == 0 && D_I <= 128, "d_I");
+};
+
+__device__ __forceinline__ void decode_item(const Params& p, int u, int& b, int& qg, int& kc) {
+  const int per = p.B * p.n_kc;
+  const int qg_rev = u / per;  // later (longer) query groups first
+  const int rem = u - qg_rev * per;
+  b = rem / p.n_kc;
+  kc = rem - b * p.n_kc;
+  qg = p.n_qg - 1 - qg_rev;
+}
+
+// Tiles [kt0, kt1) of the item; the first n_comp of them hold visible keys and need the MMA.
+template <int G>
+__device__ __forceinline__ void item_tiles(const Params& p, int qg, int kc, int& kt0, int& kt1,
+                                           int& n_comp) {
+  kt0 = kc * p.kc;
+  kt1 = min(kt0 + p.kc, p.n_kt);
+  const int i_last = min(qg * G + G, p.Lq) - 1;
+  const int t_max = i_last + (p.Lk - p.Lq);
+  const int last_visible_tile = t_max / kTileKeys;
+  n_comp = max(0, min(kt1, last_visible_tile + 1) - kt0);
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+template <int H_I, int D_I, int G>
+__global__ void __launch_bounds__(kThreads, 1)
+    indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const Params p) {
+  using C = Cfg<H_I, D_I, G>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sQ = smem + C::kOffQ;
+  uint8_t* sK = smem + C::kOffK;
+  float* sW = reinterpret_cast<float*>(smem + C::kOffW);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  uint64_t* k_full = bars;
+  uint64_t* k_empty = bars + kStages;
+  uint64_t* q_full = bars + 2 * kStages;
+  uint64_t* q_empty = q_full + 2;
+  uint64_t* acc_full = q_full + 4;
+  uint64_t* acc_empty = q_full + 6;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], 1);
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], C::kEpiWorkers);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 2) tmem_alloc(tmem_slot, C::kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      int ks = 0;
+      uint32_t kph = 0;
+      int qi = 0;
+      for (int u = blockIdx.x; u < p.n_items; u += gridDim.x) {
+        int b, qg, kc, kt0, kt1, n_comp;
+        decode_item(p, u, b, qg, kc);
+        item_tiles<G>(p, qg, kc, kt0, kt1, n_comp);
+        if (n_comp == 0) continue;
+        const int qb = qi & 1;
+        const uint32_t qph = (qi >> 1) & 1;
+        if (!mbar_wait(&q_empty[qb], qph ^ 1, abort_flag, 1)) goto done;
+        mbar_arrive_expect_tx(&q_full[qb], C::kQBytes);
+        tma_load_2d(sQ + qb * ((C::kQBytes + 1023) / 1024) * 1024, &tm_q, &q_full[qb], 0,
+                    (b * p.Lq + qg * G) * H_I);
+        for (int tt = 0; tt < n_comp; ++tt) {
+          if (!mbar_wait(&k_empty[ks], kph ^ 1, abort_flag, 2)) goto done;
+          mbar_arrive_expect_tx(&k_full[ks], C::kKBytes);
+          tma_load_2d(sK + ks * C::kKBytes, &tm_k, &k_full[ks], 0,
+                      b * p.Lk + (kt0 + tt) * kTileKeys);
+          if (++ks == kStages) {
+            ks = 0;
+            kph ^= 1;
+          }
+        }
+        ++qi;
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int ks = 0;
+      uint32_t kph = 0;
+      int ab = 0;
+      uint32_t aph = 0;
+      int qi = 0;
+      for (int u = blockIdx.x; u < p.n_items; u += gridDim.x) {
+        int b, qg, kc, kt0, kt1, n_comp;
+        decode_item(p, u, b, qg, kc);
+        item_tiles<G>(p, qg, kc, kt0, kt1, n_comp);
+        if (n_comp == 0) continue;
+        const int qb = qi & 1;
+        const uint32_t qph = (qi >> 1) & 1;
+        if (!mbar_wait(&q_full[qb], qph, abort_flag, 3)) goto done;
+        const uint32_t q_addr = smem_u32(sQ + qb * ((C::kQBytes + 1023) / 1024) * 1024);
+        for (int tt = 0; tt < n_comp; ++tt) {
+          if (!mbar_wait(&acc_empty[ab], aph ^ 1, abort_flag, 4)) goto done;
+          if (!mbar_wait(&k_full[ks], kph, abort_flag, 5)) goto done;
+          tc_fence_after();
+          const uint32_t k_addr = smem_u32(sK + ks * C::kKBytes);
+          const uint32_t d_tmem = tmem_base + ab * C::N;
+#pragma unroll
+          for (int kk = 0; kk < D_I / 32; ++kk) {
+            const uint64_t adesc = make_smem_desc(k_addr + kk * 32, 16, 8 * D_I, C::kSwizzle);
+            const uint64_t bdesc = make_smem_desc(q_addr + kk * 32, 16, 8 * D_I, C::kSwizzle);
+            mma_f8f6f4_ss(d_tmem, adesc, bdesc, C::kIdesc, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(&k_empty[ks]);
+          mma_commit(&acc_full[ab]);
+          if (++ks == kStages) {
+            ks = 0;
+            kph ^= 1;
+          }
+          ab ^= 1;
+          if (ab == 0) aph ^= 1;
+        }
+        mma_commit(&q_empty[qb]);
+        ++qi;
+      }
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------------ epilogue
+    const int e = threadIdx.x - 128;  // 0..255
+    const int wg = e >> 7;            // warpgroup 0 / 1
+    const int sp = warp & 3;          // TMEM sub-partition this warp may access
+    const int row = sp * 32 + lane;   // accumulator row = key within the tile
+    const bool worker = C::kSplitWG || wg == 0;
+    bool ok = true;
+    int ab = 0;
+    uint32_t aph = 0;
+    int it = 0;
+    for (int u = blockIdx.x; u < p.n_items; u += gridDim.x, ++it) {
+      int b, qg, kc, kt0, kt1, n_comp;
+      decode_item(p, u, b, qg, kc);
+      item_tiles<G>(p, qg, kc, kt0, kt1, n_comp);
+      const int i0 = qg * G;
+      float* wbuf = sW + (it & 1) * C::N;
+      for (int x = e; x < C::N; x += 256) {
+        const int i = i0 + x / H_I;
+        wbuf[x] = (i < p.Lq) ? p.w[(static_cast<size_t>(b) * p.Lq + i) * H_I + (x % H_I)] : 0.f;
+      }
+      named_bar_sync(1, 256);
+      const size_t row_base = static_cast<size_t>(b) * p.Lq;
+      for (int tt = 0; tt < n_comp; ++tt) {
+        if (!worker || !ok) continue;
+        const bool got = mbar_wait(&acc_full[ab], aph, abort_flag, 6);
+        if (!__all_sync(0xFFFFFFFFu, got)) {  // tcgen05.ld below is warp-collective
+          ok = false;  // keep reaching the named barriers; skip the remaining work
+          continue;
+        }
+        tc_fence_after();
+        float acc[C::kQPerWG];
+#pragma unroll
+        for (int g = 0; g < C::kQPerWG; ++g) acc[g] = 0.f;
+        const int col0 = wg * C::kColsPerWG;  // 0 when not split
+        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(sp * 32) << 16) + ab * C::N + col0;
+#pragma unroll
+        for (int ch = 0; ch < C::kColsPerWG / 32; ++ch) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(taddr + ch * 32, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const int col = ch * 32 + c;
+            acc[col / H_I] = fmaf(wbuf[col0 + col], fmaxf(__uint_as_float(v[c]), 0.f), acc[col / H_I]);
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&acc_empty[ab]);
+        ab ^= 1;
+        if (ab == 0) aph ^= 1;
+        const int s = (kt0 + tt) * kTileKeys + row;
+        if (s < p.Lk) {
+#pragma unroll
+          for (int g = 0; g < C::kQPerWG; ++g) {
+            const int i = i0 + wg * C::kQPerWG * (C::kSplitWG ? 1 : 0) + g;
+            if (i < p.Lq) {
+              const int t = i + p.Lk - p.Lq;
+              p.scores[(row_base + i) * p.Lk + s] = (s <= t) ? acc[g] : -INFINITY;
+            }
+          }
+        }
+      }
+      // keep the accumulator ring in step on the idle warpgroup
+      if (!worker) {
+        for (int tt = 0; tt < n_comp; ++tt) {
+          ab ^= 1;
+          if (ab == 0) aph ^= 1;
+        }
+      }
+      // fully masked tiles: no MMA, just -inf
+      for (int kt = kt0 + n_comp; ok && kt < kt1; ++kt) {
+        for (int x = e; x < G * kTileKeys; x += 256) {
+          const int i = i0 + x / kTileKeys;
+          const int s = kt * kTileKeys + (x % kTileKeys);
+          if (i < p.Lq && s < p.Lk) p.scores[(row_base + i) * p.Lk + s] = -INFINITY;
+        }
+      }
+    }
+  }
+done:
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
+}  // namespace indexer
+}  // namespace dsa
