@@ -52,7 +52,11 @@ def _whole_tensor_properties(wl, res):
             assert bool(((ixc <= t) | ~valid).all())
             d = ixc[:, 1:] - ixc[:, :-1]
             assert bool(((d > 0) | ~valid[:, 1:]).all())
-            sel = torch.zeros_like(sc, dtype=torch.bool).scatter_(1, ixc, valid)
+            # mark the selected positions; empty slots go to a spare column so that they can
+            # never overwrite a real position's mark
+            tgt = torch.where(valid, ix, torch.full_like(ix, Lk))
+            sel = torch.zeros(sc.shape[0], Lk + 1, dtype=torch.bool, device=sc.device)
+            sel = sel.scatter_(1, tgt, True)[:, :Lk]
             gathered = torch.gather(sc, 1, ixc)
             cut = torch.where(valid, gathered, torch.full_like(gathered, float("inf"))).min(1).values
             unsel = vis & ~sel
