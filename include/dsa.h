@@ -137,6 +137,30 @@ dsa_status dsa_indexer_kl(const float* scores, const int32_t* idx, const float* 
                           size_t ws_bytes, dsa_stream_t stream);
 
 /*
+ * The indexer loss of dsa_indexer_kl for callers that cannot hand the library any scratch
+ * memory.  The pages have no counterpart to this entry point; it exists only for how memory
+ * is provided.  Some callers cannot allocate device memory when they call in: a serving
+ * runtime that reserves all of HBM up front and forbids further cudaMalloc, a plugin that
+ * only receives pointers to its inputs and outputs, or a latency-critical thread that must
+ * avoid the device-wide synchronisation cudaMalloc and cudaFree can cause.  This variant
+ * takes the same arguments minus ws/ws_bytes and allocates nothing: when loss_per_query is
+ * NULL, the per-row KL terms go to a fixed 4 MiB array inside the library (one per GPU that
+ * loads it, held until the process exits).
+ *   - At most 1048576 query rows (B * Lq); larger sizes return DSA_ERR_UNSUPPORTED without
+ *     launching anything.
+ *   - The first call on each device looks up that array's device address (with the device
+ *     current); make that first call before any stream capture.
+ *   - Every call shares the one array and leaves its rows in it; each call writes every row
+ *     it reads, so nothing needs clearing, but calls whose kernels overlap on the GPU (on
+ *     different streams, or from different host threads) race on it.  Serialise them.
+ *   - No cudaMalloc, cudaFree or other allocating routine is called.
+ * Results are identical to dsa_indexer_kl on the same inputs.
+ */
+dsa_status dsa_indexer_kl_noalloc(const float* scores, const int32_t* idx, const float* p_sel,
+                                  int B, int Lq, int Lk, int k, float* loss,
+                                  float* loss_per_query, dsa_stream_t stream);
+
+/*
  * Waits for `stream`, then returns and clears the device status word that kernels set
  * when a bounded wait expires (DSA_ERR_TIMEOUT) - DSA_OK if none did.  Synchronising;
  * meant for tests and diagnostics.  Returns DSA_ERR_CUDA if the stream itself failed.

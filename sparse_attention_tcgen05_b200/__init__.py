@@ -17,13 +17,15 @@ from . import build as _build
 
 __all__ = [
     "DsaError", "load", "dsa_status_str", "dsa_version", "dsa_workspace_bytes", "dsa_indexer",
-    "dsa_topk", "dsa_sparse_mla_fwd", "dsa_indexer_kl", "dsa_last_device_status",
+    "dsa_topk", "dsa_sparse_mla_fwd", "dsa_indexer_kl", "dsa_indexer_kl_noalloc",
+    "dsa_last_device_status",
     "DSA_OP_INDEXER", "DSA_OP_TOPK", "DSA_OP_SPARSE_MLA_FWD", "DSA_OP_INDEXER_KL", "EXPORTED",
 ]
 
 DSA_OP_INDEXER, DSA_OP_TOPK, DSA_OP_SPARSE_MLA_FWD, DSA_OP_INDEXER_KL = 0, 1, 2, 3
 EXPORTED = ("dsa_status_str", "dsa_version", "dsa_workspace_bytes", "dsa_indexer", "dsa_topk",
-            "dsa_sparse_mla_fwd", "dsa_indexer_kl", "dsa_last_device_status")
+            "dsa_sparse_mla_fwd", "dsa_indexer_kl", "dsa_indexer_kl_noalloc",
+            "dsa_last_device_status")
 
 
 class DsaError(RuntimeError):
@@ -54,9 +56,10 @@ def load(rebuild: bool = False) -> ctypes.CDLL:
         lib.dsa_sparse_mla_fwd.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, f32, vp,
                                            vp, vp, vp, sz, vp]
         lib.dsa_indexer_kl.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, vp, vp, sz, vp]
+        lib.dsa_indexer_kl_noalloc.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, vp, vp]
         lib.dsa_last_device_status.argtypes = [vp]
         for name in ("dsa_indexer", "dsa_topk", "dsa_sparse_mla_fwd", "dsa_indexer_kl",
-                     "dsa_last_device_status"):
+                     "dsa_indexer_kl_noalloc", "dsa_last_device_status"):
             getattr(lib, name).restype = i32
         _lib = lib
     return _lib
@@ -175,6 +178,25 @@ def dsa_indexer_kl(scores: torch.Tensor, idx: torch.Tensor, p_sel: torch.Tensor,
     _raise("dsa_indexer_kl",
            load().dsa_indexer_kl(_ptr(scores), _ptr(idx), _ptr(p_sel), B, Lq, Lk, k, _ptr(loss),
                                  _ptr(loss_per_query), wsp, wsb, _stream(stream)))
+
+
+def dsa_indexer_kl_noalloc(scores: torch.Tensor, idx: torch.Tensor, p_sel: torch.Tensor,
+                           loss: torch.Tensor, loss_per_query: torch.Tensor | None = None,
+                           stream=None) -> None:
+    """dsa_indexer_kl for callers that cannot provide scratch memory: the per-row terms use a
+    fixed array inside the library (at most 1048576 rows; calls that overlap on the GPU race
+    on it)."""
+    B, Lq, Lk = scores.shape
+    k = idx.shape[2]
+    _check(scores, "scores", torch.float32, (B, Lq, Lk))
+    _check(idx, "idx", torch.int32, (B, Lq, k))
+    _check(p_sel, "p_sel", torch.float32, (B, Lq, k))
+    _check(loss, "loss", torch.float32, (1,))
+    if loss_per_query is not None:
+        _check(loss_per_query, "loss_per_query", torch.float32, (B, Lq))
+    _raise("dsa_indexer_kl_noalloc",
+           load().dsa_indexer_kl_noalloc(_ptr(scores), _ptr(idx), _ptr(p_sel), B, Lq, Lk, k,
+                                         _ptr(loss), _ptr(loss_per_query), _stream(stream)))
 
 
 def dsa_last_device_status(stream=None) -> int:

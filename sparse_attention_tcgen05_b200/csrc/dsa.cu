@@ -248,6 +248,35 @@ dsa_status launch_mla(const void* q, const void* kv, const int32_t* idx, int B, 
   return DSA_OK;
 }
 
+// ------------------------------------------------------------------------------ indexer KL without
+// caller scratch.  The per-row KL terms go to a fixed device array that every GPU loading the
+// library holds until the process exits; its address is looked up once per device.
+constexpr int kKlNoAllocMaxRows = 1 << 20;  // 4 MiB of fp32 per device
+static __device__ __align__(256) float g_kl_rows_scratch[kKlNoAllocMaxRows];
+
+struct KlScratch {
+  std::once_flag once;
+  float* ptr = nullptr;
+  cudaError_t err = cudaSuccess;
+};
+KlScratch g_kl_scratch[kMaxDevices];
+
+// Device address of g_kl_rows_scratch on the current device.  The name itself is only a host
+// stand-in, so the address must come from cudaGetSymbolAddress with that device current.
+dsa_status kl_scratch_for_current_device(float** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DSA_ERR_CUDA;
+  KlScratch& s = g_kl_scratch[dev];
+  std::call_once(s.once, [&s]() {
+    void* p = nullptr;
+    s.err = cudaGetSymbolAddress(&p, g_kl_rows_scratch);
+    s.ptr = static_cast<float*>(p);
+  });
+  if (s.err != cudaSuccess || s.ptr == nullptr) return DSA_ERR_CUDA;
+  *out = s.ptr;
+  return DSA_OK;
+}
+
 }  // namespace
 
 // ================================================================================ C ABI
@@ -380,6 +409,32 @@ dsa_status dsa_indexer_kl(const float* scores, const int32_t* idx, const float* 
   DeviceInfo dev;
   const dsa_status ds = current_device(dev);
   if (ds != DSA_OK) return ds;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  dsa::kl::kl_rows_kernel<<<static_cast<unsigned>(rows), dsa::kl::kRowThreads, 0, st>>>(
+      scores, idx, p_sel, Lk, k, per_row);
+  if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
+  dsa::kl::kl_sum_kernel<<<1, dsa::kl::kSumThreads, 0, st>>>(per_row, static_cast<int>(rows), loss);
+  return launch_result();
+}
+
+dsa_status dsa_indexer_kl_noalloc(const float* scores, const int32_t* idx, const float* p_sel,
+                                  int B, int Lq, int Lk, int k, float* loss,
+                                  float* loss_per_query, dsa_stream_t stream) {
+  if (!scores || !idx || !p_sel || !loss) return DSA_ERR_INVALID_ARG;
+  if (B <= 0 || Lq <= 0 || Lk <= 0 || Lq > Lk || k <= 0) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(scores) || !aligned16(idx) || !aligned16(p_sel) || (reinterpret_cast<uintptr_t>(loss) & 3u))
+    return DSA_ERR_INVALID_ARG;
+  const long rows = static_cast<long>(B) * Lq;
+  if (rows > kKlNoAllocMaxRows) return DSA_ERR_UNSUPPORTED;
+  DeviceInfo dev;
+  const dsa_status ds = current_device(dev);
+  if (ds != DSA_OK) return ds;
+  float* per_row = loss_per_query;
+  if (per_row == nullptr) {
+    const dsa_status ss = kl_scratch_for_current_device(&per_row);
+    if (ss != DSA_OK) return ss;
+  }
+  // Every row's term is written before the sum reads it, so the shared array needs no clearing.
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   dsa::kl::kl_rows_kernel<<<static_cast<unsigned>(rows), dsa::kl::kRowThreads, 0, st>>>(
       scores, idx, p_sel, Lk, k, per_row);
