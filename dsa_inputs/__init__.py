@@ -149,6 +149,10 @@ WORKLOADS = {
                                576, 512, 1.0 / math.sqrt(192.0), emit_p=True),
     "decode_128k": Workload("decode_128k", 0xD5A0 + 6, 32, 1, 131072, 64, 128, 16, 2048, 128, 576, 512,
                             1.0 / math.sqrt(192.0)),
+    # a 4K-token prefill with the full dims: small enough for counter captures (about 1 GB on
+    # the device) while its inputs still exceed the 126 MB L2
+    "prefill_1x4k": Workload("prefill_1x4k", 0xD5A0 + 8, 1, 4096, 4096, 64, 128, 16, 2048, 128, 576,
+                             512, 1.0 / math.sqrt(192.0)),
 }
 
 

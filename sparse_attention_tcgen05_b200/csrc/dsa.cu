@@ -14,6 +14,7 @@
 #include "indexer_kl.cuh"
 #include "ptx.cuh"
 #include "sparse_mla.cuh"
+#include "sparse_mla_pair.cuh"
 #include "status.cuh"
 #include "topk.cuh"
 
@@ -171,7 +172,8 @@ dsa_status launch_topk(const float* scores, int32_t* idx, int B, int Lq, int Lk,
 int topk_cluster_size(int rows, int Lk, int sms) {
   int c = 1;
   while (c < 8 && (Lk + c - 1) / c > dsa::topk::kMaxSlice) c *= 2;
-  while (c < 8 && static_cast<long>(rows) * c < sms && (Lk + 2 * c - 1) / (2 * c) >= 4096) c *= 2;
+  // more CTAs per row only while the doubled grid still runs in one wave
+  while (c < 8 && static_cast<long>(rows) * 2 * c <= sms && (Lk + 2 * c - 1) / (2 * c) >= 4096) c *= 2;
   return c;
 }
 
@@ -232,13 +234,34 @@ dsa_status launch_mla(const void* q, const void* kv, const int32_t* idx, int B, 
   if (!encode_2d(&tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, D_QK, static_cast<uint64_t>(rows) * H,
                  static_cast<uint64_t>(D_QK) * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
     return DSA_ERR_CUDA;
-  auto kern = dsa::mla::sparse_mla_kernel<D_QK, D_V>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) !=
-      cudaSuccess)
-    return DSA_ERR_CUDA;
   const long grid = static_cast<long>(rows) * Cfg::kNdv * sp.n_split;
   if (grid > INT32_MAX) return DSA_ERR_UNSUPPORTED;
-  kern<<<static_cast<unsigned>(grid), dsa::mla::kThreads, Cfg::kSmemBytes, stream>>>(tm_q, p);
+  if constexpr (D_QK == dsa::mla_pair::kDQK && D_V == dsa::mla_pair::kDV) {
+    // cluster of two CTAs per (row, split): QK dims and value dims split between them
+    auto kern = dsa::mla_pair::sparse_mla_pair_kernel;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             dsa::mla_pair::kSmemBytes) != cudaSuccess)
+      return DSA_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(dsa::mla_pair::kThreads);
+    cfg.dynamicSmemBytes = dsa::mla_pair::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, tm_q, p) != cudaSuccess) return DSA_ERR_CUDA;
+  } else {
+    auto kern = dsa::mla::sparse_mla_kernel<D_QK, D_V>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) !=
+        cudaSuccess)
+      return DSA_ERR_CUDA;
+    kern<<<static_cast<unsigned>(grid), dsa::mla::kThreads, Cfg::kSmemBytes, stream>>>(tm_q, p);
+  }
   if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
   if (sp.n_split > 1) {
     dsa::mla::combine_kernel<D_V><<<rows * H, 128, 0, stream>>>(
