@@ -9,8 +9,8 @@
 // so each CTA gathers only its own dims of every selected entry (each latent byte is read
 // once per pair) and holds only its slice of Q.  Each CTA computes a partial S over its dims
 // on the tensor cores (tcgen05 kind::f16, heads on the 128 TMEM lanes), ships the 128 x 32
-// fp32 partial to its peer with one asynchronous shared-to-shared bulk copy per block
-// (completing on the peer's mbarrier), and adds the peer's partial: both CTAs then hold the
+// fp32 partial to its peer with asynchronous remote stores (st.async, counted on the peer's
+// mbarrier), and adds the peer's partial: both CTAs then hold the
 // same full S (fp32 addition commutes), run the same online softmax and accumulate O for
 // their own 256 value dims in TMEM.
 //
@@ -38,7 +38,7 @@ using mla::named_bar_sync;
 
 constexpr int kBN = 32;          // selected entries per block
 constexpr int kHalf = kBN / 2;   // columns per softmax warpgroup
-constexpr int kStages = 3;       // gather ring
+constexpr int kStages = 4;       // gather ring
 constexpr int kThreads = 416;
 constexpr int kSoftmaxThreads = 256;
 constexpr int kMmaWarp = 8;
@@ -54,8 +54,7 @@ constexpr int kOffQ = 0;
 constexpr int kOffKV = kOffQ + kMaxBoxes * kQBox;
 constexpr int kOffP = kOffKV + kStages * kKvStage;
 constexpr int kOffX = kOffP + 2 * kPBytes;     // 2 slots received from the peer
-constexpr int kOffXs = kOffX + 2 * kXSlot;     // 2 slots staged for the copy to the peer
-constexpr int kOffRed = kOffXs + 2 * kXSlot;   // [8 warps][16] p partial sums
+constexpr int kOffRed = kOffX + 2 * kXSlot;    // [8 warps][16] p partial sums
 constexpr int kOffMax = kOffRed + 8 * 16 * 4;  // [2][128] row-max exchange
 constexpr int kOffL = kOffMax + 2 * 128 * 4;   // [2][128] normaliser exchange
 constexpr int kOffBar = kOffL + 2 * 128 * 4;
@@ -93,7 +92,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sKV = smem + kOffKV;
   uint8_t* sP = smem + kOffP;
   float* sX = reinterpret_cast<float*>(smem + kOffX);
-  float* sXs = reinterpret_cast<float*>(smem + kOffXs);
   float* sRed = reinterpret_cast<float*>(smem + kOffRed);
   float* sMax = reinterpret_cast<float*>(smem + kOffMax);
   float* sL = reinterpret_cast<float*>(smem + kOffL);
@@ -104,7 +102,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* s_empty = s_full + 2;           // [2] 256 softmax arrivals
   uint64_t* p_full = s_full + 4;            // [2] 256 softmax arrivals
   uint64_t* o_done = s_full + 6;            // [2] MMA commit (PV of blocks q, q % 2)
-  uint64_t* x_full = s_full + 8;            // [2] own expect_tx + the peer's copy bytes
+  uint64_t* x_full = s_full + 8;            // [2] own expect_tx + the peer's stored bytes
   uint64_t* q_full = s_full + 10;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
@@ -145,7 +143,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (warp == kMmaWarp) tmem_alloc(tmem_slot, kTmemCols);
   tc_fence_before();
-  // the peer's barriers must be initialised before any copy completes on them
+  // the peer's barriers must be initialised before any remote store completes on them
   cluster_barrier();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
@@ -246,11 +244,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int col0 = wg * kHalf;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t o_cols = static_cast<uint32_t>(wg * (kDvCta / 2));
-    // Exchange of partial S.  Slot q % 2 of this CTA's staging buffer is copied into slot q % 2
-    // of the peer's receive buffer.  Two slots suffice without a back-signal: before this CTA
-    // reuses a slot (step q + 2) it has received the peer's copy of step q + 1, which the peer
-    // issues only after it consumed step q, and that copy could only complete after this CTA's
-    // step-q copy had landed.
+    // Exchange of partial S: at step q every thread stores its 16 values into slot q % 2 of the
+    // peer's receive buffer (row h = 128 B, 16-byte chunk j kept at chunk j ^ (h % 8) so that a
+    // warp's accesses spread over all banks).  Two slots suffice without a back-signal: before
+    // this CTA reuses a slot (step q + 2) it has received all of the peer's step q + 1 stores,
+    // which the peer issues only after it consumed step q.
     const uint32_t peer_recv = map_to_rank(smem_u32(sX), peer);
     const uint32_t peer_x_full = map_to_rank(smem_u32(x_full), peer);
     float m_ref = -INFINITY;  // running reference max (log2 domain), identical in both halves
@@ -271,39 +269,40 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __all_sync(0xFFFFFFFFu, ok);  // TMEM accesses below are warp-collective
       uint32_t v[kHalf];
       float x[kHalf];
+      const uint32_t xrow = static_cast<uint32_t>(sb * kXSlot + h * (kBN * 4));
+      const uint32_t hsw = static_cast<uint32_t>(h & 7);
       if (ok) {
         tc_fence_after();
         tmem_ld_32x32b_x16(tmem_s + sb * kBN + col0 + lane_off, v);
         tmem_ld_wait();
         tc_fence_before();
         mbar_arrive(&s_empty[sb]);
-        float4* stg = reinterpret_cast<float4*>(sXs + sb * (kXSlot / 4) + h * kBN + col0);
-#pragma unroll
-        for (int c = 0; c < kHalf; c += 4)
-          stg[c / 4] = make_float4(__uint_as_float(v[c]), __uint_as_float(v[c + 1]),
-                                   __uint_as_float(v[c + 2]), __uint_as_float(v[c + 3]));
-        fence_proxy_async_smem();  // the bulk copy reads the staged rows through the async proxy
         if (threadIdx.x == 0) mbar_arrive_expect_tx(&x_full[sb], kXSlot);
+#pragma unroll
+        for (int i = 0; i < kHalf / 4; ++i) {
+          const uint32_t j = static_cast<uint32_t>(wg * 4 + i);
+          st_async_v4(peer_recv + xrow + ((j ^ hsw) << 4), __uint_as_float(v[4 * i]),
+                      __uint_as_float(v[4 * i + 1]), __uint_as_float(v[4 * i + 2]),
+                      __uint_as_float(v[4 * i + 3]), peer_x_full + sb * 8);
+        }
       } else {
 #pragma unroll
         for (int c = 0; c < kHalf; ++c) v[c] = 0u;
       }
-      named_bar_sync(kBarSoftmax, kSoftmaxThreads);  // every row staged
-      if (ok && threadIdx.x == 0)
-        bulk_copy_to_peer(peer_recv + sb * kXSlot, smem_u32(sXs + sb * (kXSlot / 4)), kXSlot,
-                          peer_x_full + sb * 8);
       if (ok && !mbar_wait_cluster(&x_full[sb], ph, abort_flag, 47)) ok = false;
       ok = __all_sync(0xFFFFFFFFu, ok);
       float bm = -INFINITY;
       {
-        const float4* theirs = reinterpret_cast<const float4*>(sX + sb * (kXSlot / 4) + h * kBN + col0);
+        const uint8_t* mine = reinterpret_cast<const uint8_t*>(sX) + xrow;
 #pragma unroll
-        for (int c = 0; c < kHalf; c += 4) {
-          const float4 u = ok ? theirs[c / 4] : make_float4(0.f, 0.f, 0.f, 0.f);
-          x[c] = __uint_as_float(v[c]) + u.x;
-          x[c + 1] = __uint_as_float(v[c + 1]) + u.y;
-          x[c + 2] = __uint_as_float(v[c + 2]) + u.z;
-          x[c + 3] = __uint_as_float(v[c + 3]) + u.w;
+        for (int i = 0; i < kHalf / 4; ++i) {
+          const uint32_t j = static_cast<uint32_t>(wg * 4 + i);
+          const float4 u = ok ? *reinterpret_cast<const float4*>(mine + ((j ^ hsw) << 4))
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+          x[4 * i] = __uint_as_float(v[4 * i]) + u.x;
+          x[4 * i + 1] = __uint_as_float(v[4 * i + 1]) + u.y;
+          x[4 * i + 2] = __uint_as_float(v[4 * i + 2]) + u.z;
+          x[4 * i + 3] = __uint_as_float(v[4 * i + 3]) + u.w;
         }
 #pragma unroll
         for (int c = 0; c < kHalf; ++c) {
