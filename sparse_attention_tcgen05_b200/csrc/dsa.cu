@@ -142,19 +142,14 @@ dsa_status launch_indexer(const void* q, const void* kk, const float* w, float* 
 }
 
 // ------------------------------------------------------------------------------ top-k
-template <int C>
+template <int C, int KPT>
 dsa_status launch_topk(const float* scores, int32_t* idx, int B, int Lq, int Lk, int k,
                        cudaStream_t stream) {
-  const int slice = (Lk + C - 1) / C;
-  const size_t smem = static_cast<size_t>(slice) * sizeof(uint32_t);
-  auto kern = dsa::topk::topk_kernel<C>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem)) != cudaSuccess)
-    return DSA_ERR_CUDA;
+  auto kern = dsa::topk::topk_kernel<C, KPT>;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(B) * Lq * C);
   cfg.blockDim = dim3(dsa::topk::kThreads);
-  cfg.dynamicSmemBytes = smem;
+  cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -163,18 +158,29 @@ dsa_status launch_topk(const float* scores, int32_t* idx, int B, int Lq, int Lk,
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (C > 1 && cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 0) != cudaSuccess)
-    return DSA_ERR_CUDA;
   if (cudaLaunchKernelEx(&cfg, kern, scores, idx, B, Lq, Lk, k) != cudaSuccess) return DSA_ERR_CUDA;
   return launch_result();
 }
 
+// Keys per CTA for a row split over c CTAs (a multiple of 4, as the kernel computes it).
+inline int topk_slice(int Lk, int c) { return (((Lk + c - 1) / c) + 3) & ~3; }
+
 int topk_cluster_size(int rows, int Lk, int sms) {
   int c = 1;
-  while (c < 8 && (Lk + c - 1) / c > dsa::topk::kMaxSlice) c *= 2;
+  while (c < 8 && topk_slice(Lk, c) > dsa::topk::kMaxSlice) c *= 2;
   // more CTAs per row only while the doubled grid still runs in one wave
-  while (c < 8 && static_cast<long>(rows) * 2 * c <= sms && (Lk + 2 * c - 1) / (2 * c) >= 4096) c *= 2;
+  while (c < 8 && static_cast<long>(rows) * 2 * c <= sms && topk_slice(Lk, 2 * c) >= 4096) c *= 2;
   return c;
+}
+
+template <int C>
+dsa_status launch_topk_c(const float* scores, int32_t* idx, int B, int Lq, int Lk, int k,
+                         cudaStream_t st) {
+  const int slice = topk_slice(Lk, C);
+  if (slice <= 4 * dsa::topk::kThreads) return launch_topk<C, 4>(scores, idx, B, Lq, Lk, k, st);
+  if (slice <= 8 * dsa::topk::kThreads) return launch_topk<C, 8>(scores, idx, B, Lq, Lk, k, st);
+  if (slice <= 16 * dsa::topk::kThreads) return launch_topk<C, 16>(scores, idx, B, Lq, Lk, k, st);
+  return launch_topk<C, 32>(scores, idx, B, Lq, Lk, k, st);
 }
 
 // ------------------------------------------------------------------------------ sparse MLA
@@ -376,17 +382,17 @@ dsa_status dsa_topk(const float* scores, int32_t* idx, int B, int Lq, int Lk, in
   if (!scores || !idx) return DSA_ERR_INVALID_ARG;
   if (B <= 0 || Lq <= 0 || Lk <= 0 || Lq > Lk || k <= 0) return DSA_ERR_INVALID_ARG;
   if (!aligned16(scores) || !aligned16(idx)) return DSA_ERR_INVALID_ARG;
-  if (k > 4096 || Lk > 8 * dsa::topk::kMaxSlice) return DSA_ERR_UNSUPPORTED;
+  if (k > 4096 || topk_slice(Lk, 8) > dsa::topk::kMaxSlice) return DSA_ERR_UNSUPPORTED;
   if (static_cast<long>(B) * Lq * 8 > INT32_MAX) return DSA_ERR_UNSUPPORTED;
   DeviceInfo dev;
   const dsa_status ds = current_device(dev);
   if (ds != DSA_OK) return ds;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   switch (topk_cluster_size(B * Lq, Lk, dev.sms)) {
-    case 1: return launch_topk<1>(scores, idx, B, Lq, Lk, k, st);
-    case 2: return launch_topk<2>(scores, idx, B, Lq, Lk, k, st);
-    case 4: return launch_topk<4>(scores, idx, B, Lq, Lk, k, st);
-    default: return launch_topk<8>(scores, idx, B, Lq, Lk, k, st);
+    case 1: return launch_topk_c<1>(scores, idx, B, Lq, Lk, k, st);
+    case 2: return launch_topk_c<2>(scores, idx, B, Lq, Lk, k, st);
+    case 4: return launch_topk_c<4>(scores, idx, B, Lq, Lk, k, st);
+    default: return launch_topk_c<8>(scores, idx, B, Lq, Lk, k, st);
   }
 }
 

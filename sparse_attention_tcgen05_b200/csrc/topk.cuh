@@ -1,12 +1,14 @@
 // Top-k selection S_t ("DeepSeek-V3.2" analysis page, sec. 1.1, eq. (2) and the S_t of eq. (4)):
 // the min(k, t+1) positions s <= t with the largest scores, ties to the smaller position.
 //
-// Radix select over order-preserving 32-bit keys, one row per cluster of C CTAs.  Each CTA
-// stages its slice of the row in shared memory once (the only HBM read), then four 8-bit
-// digit passes build warp-aggregated shared histograms; with C > 1 the C histograms are
-// summed through distributed shared memory.  The threshold key T and the number r of
-// threshold ties to keep fix the set exactly; a final ordered pass (ballot + popc prefix
-// sums) writes the selected positions in ascending order.
+// One row per cluster of C CTAs; each CTA takes a contiguous slice of the row and each of its
+// 1024 threads a contiguous run of KPT keys, held in registers as order-preserving 32-bit keys
+// (read from HBM once).  Radix select in three digit passes (11, 11, 10 bits): shared-memory
+// histograms (summed over the cluster through distributed shared memory when C > 1) give the
+// digit holding the k-th largest key; later passes only count keys that still match the
+// chosen prefix.  The threshold key T and the number r of T-ties to keep fix the set exactly.
+// Because every thread owns a contiguous run, one exclusive scan of the per-thread counts of
+// (key > T, key == T) gives every selected position's place in ascending order.
 #pragma once
 
 #include <cuda_runtime.h>
@@ -18,214 +20,221 @@ namespace topk {
 
 constexpr int kThreads = 1024;
 constexpr int kWarps = kThreads / 32;
-constexpr int kMaxSlice = 32768;  // keys per CTA held in shared memory (128 KiB)
+constexpr int kMaxKpt = 32;
+constexpr int kMaxSlice = kThreads * kMaxKpt;  // keys per CTA
 
+// Every finite or infinite score maps to a key >= 0x007FFFFF; 0 marks an empty register slot
+// and can never be selected (at least k real keys exist whenever a row is selected).
 __device__ __forceinline__ uint32_t ordered_key(float f) {
   uint32_t u = __float_as_uint(f);
   if (u == 0x80000000u) u = 0u;  // -0 ties with +0
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-__device__ __forceinline__ uint32_t cluster_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-
-__device__ __forceinline__ void cluster_sync() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
-                   : "memory");
-}
-
 __device__ __forceinline__ uint32_t ld_peer_u32(const uint32_t* local, uint32_t rank) {
-  uint32_t remote, v;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
-  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(remote) : "memory");
+  uint32_t v;
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(map_to_rank(smem_u32(local), rank))
+               : "memory");
   return v;
 }
 
-// Warp-aggregated histogram increment (all 32 lanes must call; `valid` selects contributors).
-__device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin, bool valid) {
-  const uint32_t key = valid ? bin : 0xFFFFFFFFu;
-  const uint32_t peers = __match_any_sync(0xFFFFFFFFu, key);
-  const int leader = __ffs(peers) - 1;
-  if (valid && static_cast<int>(threadIdx.x & 31) == leader) atomicAdd(&hist[bin], __popc(peers));
-}
-
-// Block-wide exclusive scan of one value per warp (result for the calling warp) + total.
-__device__ __forceinline__ uint32_t warp_offsets(uint32_t warp_total, uint32_t* scratch,
-                                                 uint32_t& block_total) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (lane == 0) scratch[warp] = warp_total;
+// Digit (of `nbins`) holding the k_rem-th largest counted key, and k_rem within that digit.
+// hist: this CTA's counts; with C > 1 the cluster's counts are summed through DSMEM.
+template <int C>
+__device__ __forceinline__ void select_digit(const uint32_t* hist, int nbins, uint32_t k_rem,
+                                             uint32_t* scan, uint32_t* result, uint32_t& digit,
+                                             uint32_t& k_out) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int per = nbins / kThreads;  // bins per thread (1 or 2), taken in descending order
+  uint32_t cnt[2] = {0, 0};
+  uint32_t mine = 0;
+  for (int i = 0; i < per; ++i) {
+    const int d = nbins - 1 - (tid * per + i);
+    uint32_t c = 0;
+    if (C > 1) {
+      for (int r = 0; r < C; ++r) c += ld_peer_u32(&hist[d], r);
+    } else {
+      c = hist[d];
+    }
+    cnt[i] = c;
+    mine += c;
+  }
+  // exclusive scan of `mine` over threads (descending digits)
+  uint32_t inc = mine;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t nb = __shfl_up_sync(0xFFFFFFFFu, inc, o);
+    if (lane >= o) inc += nb;
+  }
+  if (lane == 31) scan[warp] = inc;
   __syncthreads();
   if (warp == 0) {
-    uint32_t v = scratch[lane];
-    uint32_t inc = v;
+    const uint32_t v = scan[lane];
+    uint32_t wi = v;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      uint32_t n = __shfl_up_sync(0xFFFFFFFFu, inc, o);
-      if (lane >= o) inc += n;
+      const uint32_t nb = __shfl_up_sync(0xFFFFFFFFu, wi, o);
+      if (lane >= o) wi += nb;
     }
-    scratch[32 + lane] = inc - v;
-    if (lane == 31) scratch[64] = inc;
+    scan[32 + lane] = wi - v;
   }
   __syncthreads();
-  const uint32_t off = scratch[32 + warp];
-  block_total = scratch[64];
+  uint32_t above = scan[32 + warp] + inc - mine;  // keys in digits larger than this thread's
+  for (int i = 0; i < per; ++i) {
+    if (above < k_rem && k_rem <= above + cnt[i]) {
+      result[0] = nbins - 1 - (tid * per + i);
+      result[1] = k_rem - above;
+    }
+    above += cnt[i];
+  }
   __syncthreads();
-  return off;
+  digit = result[0];
+  k_out = result[1];
 }
 
-template <int C>
+template <int C, int KPT>
 __global__ void __launch_bounds__(kThreads, 1)
     topk_kernel(const float* __restrict__ scores, int32_t* __restrict__ idx, int B, int Lq, int Lk,
                 int k) {
-  extern __shared__ uint32_t keys[];  // [slice]
-  __shared__ uint32_t hist[2][256];
+  __shared__ uint32_t hist[2][2048];
   __shared__ uint32_t scan[72];
-  __shared__ uint32_t sel_state[4];  // [0] digit, [1] k_remaining, [2] count_gt, [3] count_eq
-  __shared__ uint32_t counts[2];     // this CTA's (count_gt, count_eq) for the output pass
+  __shared__ uint32_t result[2];
+  __shared__ uint32_t totals[2];  // this CTA's (count > T, count == T), read by later ranks
 
   const int row = blockIdx.x / C;
-  const uint32_t rank = (C > 1) ? cluster_rank() : 0u;
+  const uint32_t rank = (C > 1) ? cluster_ctarank() : 0u;
   const int i = row % Lq;
   const int t = i + Lk - Lq;
   const int n = t + 1;  // candidates s in [0, n)
   int32_t* out = idx + static_cast<size_t>(row) * k;
-  const int tid = threadIdx.x, lane = tid & 31;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
   if (n <= k) {  // every visible position is selected
     for (int x = rank * kThreads + tid; x < k; x += C * kThreads) out[x] = x < n ? x : -1;
     return;
   }
 
-  const int slice = (n + C - 1) / C;
+  // ---- this thread's keys: positions [p0, p0 + KPT) of the row, clipped to the slice
+  const int slice = (((n + C - 1) / C) + 3) & ~3;  // multiple of 4: aligned vector loads
   const int lo = min(n, static_cast<int>(rank) * slice);
   const int hi = min(n, lo + slice);
-  const int len = hi - lo;
-  const float* src = scores + static_cast<size_t>(row) * Lk + lo;
-
-  // ---- stage the slice as ordered keys; histogram of the top digit on the way
-  for (int x = tid; x < 256; x += kThreads) hist[0][x] = 0u;
-  __syncthreads();
-  const int len_r = (len + kThreads - 1) / kThreads * kThreads;
-  for (int x = tid; x < len_r; x += kThreads) {
-    uint32_t key = 0;
-    const bool v = x < len;
-    if (v) {
-      key = ordered_key(__ldg(src + x));
-      keys[x] = key;
-    }
-    hist_add(hist[0], key >> 24, v);
-  }
-
-  uint32_t prefix = 0, mask = 0;
-  uint32_t k_rem = static_cast<uint32_t>(k);
-#pragma unroll 1
-  for (int pass = 0; pass < 4; ++pass) {
-    const int shift = 24 - 8 * pass;
-    uint32_t* h = hist[pass & 1];
-    if (pass > 0) {
-      for (int x = tid; x < 256; x += kThreads) h[x] = 0u;
-      __syncthreads();
-      for (int x = tid; x < len_r; x += kThreads) {
-        const bool v = x < len && ((keys[x] & mask) == prefix);
-        const uint32_t key = x < len ? keys[x] : 0u;
-        hist_add(h, (key >> shift) & 0xFFu, v);
-      }
-    }
-    __syncthreads();
-    if (C > 1) cluster_sync();
-    // Digit holding the k_rem-th largest key among those matching the prefix.  Thread
-    // tid < 256 handles digit d = 255 - tid, so an inclusive scan over tid counts the keys
-    // whose digit is >= d.  Counts are summed over the cluster through DSMEM.
-    uint32_t cd = 0, inc = 0;
-    if (tid < 256) {
-      const uint32_t d = 255u - tid;
-      if (C > 1) {
-        for (int r = 0; r < C; ++r) cd += ld_peer_u32(&h[d], r);
-      } else {
-        cd = h[d];
-      }
-      inc = cd;
+  const int p0 = lo + tid * KPT;
+  const float* src = scores + static_cast<size_t>(row) * Lk;
+  uint32_t key[KPT];
+  const bool vec = ((reinterpret_cast<uintptr_t>(src + p0) & 15u) == 0) && (p0 + KPT <= hi);
+  if (vec) {
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t nb = __shfl_up_sync(0xFFFFFFFFu, inc, o);
-        if (lane >= o) inc += nb;
-      }
-      if (lane == 31) scan[tid >> 5] = inc;
+    for (int j = 0; j < KPT; j += 4) {
+      const float4 f = __ldg(reinterpret_cast<const float4*>(src + p0 + j));
+      key[j] = ordered_key(f.x);
+      key[j + 1] = ordered_key(f.y);
+      key[j + 2] = ordered_key(f.z);
+      key[j + 3] = ordered_key(f.w);
     }
-    __syncthreads();
-    if (tid < 256) {
-      for (int x = 0; x < (tid >> 5); ++x) inc += scan[x];
-      const uint32_t above = inc - cd;  // keys with a larger digit
-      if (above < k_rem && k_rem <= inc) {
-        sel_state[0] = 255u - tid;
-        sel_state[1] = k_rem - above;
-      }
-    }
-    __syncthreads();
-    const uint32_t d = sel_state[0];
-    k_rem = sel_state[1];
-    prefix |= d << shift;
-    mask |= 0xFFu << shift;
-  }
-  const uint32_t T = prefix;      // the threshold key
-  const uint32_t r_ties = k_rem;  // keys equal to T that are kept (>= 1)
-
-  // ---- counts of keys > T and == T in this slice, shared over the cluster
-  uint32_t my_gt = 0, my_eq = 0;
-  for (int x = tid; x < len; x += kThreads) {
-    const uint32_t key = keys[x];
-    my_gt += key > T;
-    my_eq += key == T;
-  }
+  } else {
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    my_gt += __shfl_xor_sync(0xFFFFFFFFu, my_gt, o);
-    my_eq += __shfl_xor_sync(0xFFFFFFFFu, my_eq, o);
+    for (int j = 0; j < KPT; ++j) key[j] = (p0 + j < hi) ? ordered_key(__ldg(src + p0 + j)) : 0u;
   }
-  if (tid == 0) {
-    counts[0] = 0;
-    counts[1] = 0;
-  }
-  __syncthreads();
-  if (lane == 0) {
-    atomicAdd(&counts[0], my_gt);
-    atomicAdd(&counts[1], my_eq);
+
+  // ---- pass 1: top 11 bits
+  for (int x = tid; x < 2048; x += kThreads) {
+    hist[0][x] = 0u;
+    hist[1][x] = 0u;
   }
   __syncthreads();
-  uint32_t gt_before = 0, eq_before = 0;
+#pragma unroll
+  for (int j = 0; j < KPT; ++j)
+    if (key[j]) atomicAdd(&hist[0][key[j] >> 21], 1u);
+  __syncthreads();
+  if (C > 1) cluster_barrier();
+  uint32_t d1, k1;
+  select_digit<C>(hist[0], 2048, static_cast<uint32_t>(k), scan, result, d1, k1);
+
+  // ---- pass 2: bits 10..20 of keys whose top 11 bits are d1
+#pragma unroll
+  for (int j = 0; j < KPT; ++j)
+    if (key[j] && (key[j] >> 21) == d1) atomicAdd(&hist[1][(key[j] >> 10) & 2047u], 1u);
+  __syncthreads();
+  if (C > 1) cluster_barrier();  // also: every CTA has finished reading the others' pass-1 counts
+  uint32_t d2, k2;
+  select_digit<C>(hist[1], 2048, k1, scan, result, d2, k2);
+  const uint32_t pre2 = (d1 << 11) | d2;
+
+  // ---- pass 3: bits 0..9 of keys whose top 22 bits are pre2 (hist[0] is free again)
+  for (int x = tid; x < 1024; x += kThreads) hist[0][x] = 0u;
+  __syncthreads();
+#pragma unroll
+  for (int j = 0; j < KPT; ++j)
+    if (key[j] && (key[j] >> 10) == pre2) atomicAdd(&hist[0][key[j] & 1023u], 1u);
+  __syncthreads();
+  if (C > 1) cluster_barrier();
+  uint32_t d3, r_ties;
+  select_digit<C>(hist[0], 1024, k2, scan, result, d3, r_ties);
+  const uint32_t T = (pre2 << 10) | d3;  // the threshold key; r_ties keys equal to it are kept
+
+  // ---- output: one exclusive scan of (count > T, count == T) in position order
+  uint32_t gt = 0, eq = 0;
+#pragma unroll
+  for (int j = 0; j < KPT; ++j) {
+    gt += key[j] > T;
+    eq += key[j] == T;
+  }
+  uint32_t igt = gt, ieq = eq;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t a = __shfl_up_sync(0xFFFFFFFFu, igt, o);
+    const uint32_t b2 = __shfl_up_sync(0xFFFFFFFFu, ieq, o);
+    if (lane >= o) {
+      igt += a;
+      ieq += b2;
+    }
+  }
+  if (lane == 31) {
+    scan[warp] = igt;
+    scan[32 + warp] = ieq;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const uint32_t vg = scan[lane], ve = scan[32 + lane];
+    uint32_t wsum_g = vg, wsum_e = ve;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t a = __shfl_up_sync(0xFFFFFFFFu, wsum_g, o);
+      const uint32_t b2 = __shfl_up_sync(0xFFFFFFFFu, wsum_e, o);
+      if (lane >= o) {
+        wsum_g += a;
+        wsum_e += b2;
+      }
+    }
+    __syncwarp();
+    scan[lane] = wsum_g - vg;  // exclusive offsets of each warp
+    scan[32 + lane] = wsum_e - ve;
+    if (lane == 31) {
+      totals[0] = wsum_g;
+      totals[1] = wsum_e;
+    }
+  }
+  __syncthreads();
+  uint32_t gt_before = scan[warp] + igt - gt;
+  uint32_t eq_before = scan[32 + warp] + ieq - eq;
   if (C > 1) {
-    cluster_sync();
+    cluster_barrier();  // every CTA's totals are written
     for (uint32_t r = 0; r < rank; ++r) {
-      gt_before += ld_peer_u32(&counts[0], r);
-      eq_before += ld_peer_u32(&counts[1], r);
+      gt_before += ld_peer_u32(&totals[0], r);
+      eq_before += ld_peer_u32(&totals[1], r);
     }
-    cluster_sync();  // no CTA leaves while a peer may still read its counters
+    cluster_barrier();  // no CTA leaves while a peer may still read its shared memory
   }
-  const uint32_t sel_before = gt_before + min(eq_before, r_ties);
-
-  // ---- ordered output pass
-  uint32_t run_eq = 0, run_sel = 0;
-  for (int base = 0; base < len; base += kThreads) {
-    const int x = base + tid;
-    const uint32_t key = x < len ? keys[x] : 0u;
-    const bool is_gt = x < len && key > T;
-    const bool is_eq = x < len && key == T;
-    const uint32_t lt = (1u << lane) - 1u;
-    const uint32_t b_eq = __ballot_sync(0xFFFFFFFFu, is_eq);
-    uint32_t eq_total;
-    const uint32_t eq_off = warp_offsets(__popc(b_eq), scan, eq_total);
-    const uint32_t eq_rank = eq_before + run_eq + eq_off + __popc(b_eq & lt);
-    const bool sel = is_gt || (is_eq && eq_rank < r_ties);
-    const uint32_t b_sel = __ballot_sync(0xFFFFFFFFu, sel);
-    uint32_t sel_total;
-    const uint32_t sel_off = warp_offsets(__popc(b_sel), scan, sel_total);
-    const uint32_t pos = sel_before + run_sel + sel_off + __popc(b_sel & lt);
-    if (sel && pos < static_cast<uint32_t>(k)) out[pos] = lo + x;
-    run_eq += eq_total;
-    run_sel += sel_total;
+  uint32_t pos = gt_before + min(eq_before, r_ties);
+  uint32_t eq_rank = eq_before;
+#pragma unroll
+  for (int j = 0; j < KPT; ++j) {
+    bool sel = key[j] > T;
+    if (key[j] == T) {
+      sel = eq_rank < r_ties;
+      ++eq_rank;
+    }
+    if (sel && pos < static_cast<uint32_t>(k)) out[pos++] = p0 + j;
   }
 }
 
