@@ -217,6 +217,7 @@ dsa_status launch_mla(const void* q, const void* kv, const int32_t* idx, int B, 
   const int rows = B * Lq;
   const MlaSplit sp = mla_split(rows, k, Cfg::kNdv, sms, p_sel != nullptr);
   dsa::mla::Params p{};
+  p.q = static_cast<const __nv_bfloat16*>(q);
   p.kv = static_cast<const __nv_bfloat16*>(kv);
   p.idx = idx;
   p.out = static_cast<__nv_bfloat16*>(out);
@@ -236,14 +237,18 @@ dsa_status launch_mla(const void* q, const void* kv, const int32_t* idx, int B, 
     p.part_o = static_cast<float*>(ws);
     p.part_lse = p.part_o + static_cast<size_t>(sp.n_split) * rows * H * D_V;
   }
-  CUtensorMap tm_q;
-  if (!encode_2d(&tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, D_QK, static_cast<uint64_t>(rows) * H,
-                 static_cast<uint64_t>(D_QK) * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
-    return DSA_ERR_CUDA;
   const long grid = static_cast<long>(rows) * Cfg::kNdv * sp.n_split;
   if (grid > INT32_MAX) return DSA_ERR_UNSUPPORTED;
   if constexpr (D_QK == dsa::mla_pair::kDQK && D_V == dsa::mla_pair::kDV) {
     // cluster of two CTAs per (row, split): QK dims and value dims split between them
+    // kv as [B * Lk rows, 576 dims]: one-row boxes of 64 dims (SW128) and of the 32 rope dims
+    // (SW64) for the row gathers
+    CUtensorMap tm_main, tm_rope;
+    if (!encode_2d(&tm_main, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kv, D_QK, static_cast<uint64_t>(B) * Lk,
+                   static_cast<uint64_t>(D_QK) * 2, 64, 1, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_2d(&tm_rope, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kv, D_QK, static_cast<uint64_t>(B) * Lk,
+                   static_cast<uint64_t>(D_QK) * 2, 32, 1, CU_TENSOR_MAP_SWIZZLE_64B))
+      return DSA_ERR_CUDA;
     auto kern = dsa::mla_pair::sparse_mla_pair_kernel;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              dsa::mla_pair::kSmemBytes) != cudaSuccess)
@@ -260,8 +265,12 @@ dsa_status launch_mla(const void* q, const void* kv, const int32_t* idx, int B, 
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, kern, tm_q, p) != cudaSuccess) return DSA_ERR_CUDA;
+    if (cudaLaunchKernelEx(&cfg, kern, tm_main, tm_rope, p) != cudaSuccess) return DSA_ERR_CUDA;
   } else {
+    CUtensorMap tm_q;
+    if (!encode_2d(&tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, D_QK, static_cast<uint64_t>(rows) * H,
+                   static_cast<uint64_t>(D_QK) * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+      return DSA_ERR_CUDA;
     auto kern = dsa::mla::sparse_mla_kernel<D_QK, D_V>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) !=
         cudaSuccess)
@@ -406,7 +415,7 @@ dsa_status dsa_sparse_mla_fwd(const void* q_bf16, const void* kv_bf16, const int
   if (!aligned16(q_bf16) || !aligned16(kv_bf16) || !aligned16(idx) || !aligned16(out_bf16) ||
       (lse && !aligned16(lse)) || (p_sel && !aligned16(p_sel)))
     return DSA_ERR_INVALID_ARG;
-  if (H > 128 || k > 65536) return DSA_ERR_UNSUPPORTED;
+  if (H > 128 || k > 65536 || static_cast<long>(B) * Lk >= INT32_MAX) return DSA_ERR_UNSUPPORTED;
   if (static_cast<long>(B) * Lq * H * 2 * 8 > INT32_MAX) return DSA_ERR_UNSUPPORTED;
   DeviceInfo dev;
   const dsa_status ds = current_device(dev);

@@ -36,6 +36,7 @@ constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleLog2 = 8.0f;
 
 struct Params {
+  const __nv_bfloat16* q;  // [rows][H][d_qk] (read directly by the 576-d pair kernel)
   const __nv_bfloat16* kv;
   const int32_t* idx;
   __nv_bfloat16* out;   // final output (n_split == 1)
