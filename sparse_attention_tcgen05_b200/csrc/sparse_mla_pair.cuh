@@ -25,10 +25,10 @@
 //                  take turns by block (warp w always refills stage w).
 //   MMA thread     polls: S(j) = Q K_j^T as soon as block j and an S buffer are free;
 //                  O += P(i) V_i as soon as P(i) is written (never waits behind a late gather)
-//   softmax        two warpgroups on the same 128 TMEM lanes (thread = head row), each owning
-//                  16 of the block's 32 columns.  Iteration q loads S(q+1) and ships it to the
-//                  peer one block ahead, then adds the peer's part of S(q), combines the two
-//                  half-row maxima, runs the online softmax with lazy rescaling and writes P(q).
+//   softmax        two warpgroups on the same 128 TMEM lanes (thread = head row) take turns by
+//                  block, so two blocks are in flight: each loads its partial S, ships it to the
+//                  peer, adds the peer's part, settles the block's per-row reference max with
+//                  the other group (the only serial link), and writes P.  See the softmax role.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -48,8 +48,7 @@ constexpr int kBN = 32;             // selected entries per block
 constexpr int kStages = 6;          // gather ring depth (a multiple of kGatherWarps)
 constexpr int kRecvSlots = 4;       // partial-S receive slots (see the exchange argument below)
 constexpr int kThreads = 480;       // warps 0-7 softmax, 8 MMA, 9-14 gather
-constexpr int kSoftmaxThreads = 256;
-constexpr int kHalf = 16;           // S columns per softmax warpgroup
+constexpr int kSoftmaxThreads = 256;  // two warpgroups taking turns by block
 constexpr int kMmaWarp = 8;
 constexpr int kGatherWarp0 = 9;
 constexpr int kGatherWarps = 6;
@@ -64,11 +63,11 @@ constexpr int kOffKV = 0;
 constexpr int kOffX = kOffKV + kStages * kKvStage;  // [kRecvSlots] the peer's partials
 constexpr int kOffXs = kOffX + kRecvSlots * kXSlot; // [2] own partials staged for the bulk copy
 constexpr int kOffP = kOffXs + 2 * kXSlot;
-constexpr int kOffRed = kOffP + 2 * kPBytes;   // [2][8 warps][16] p partial sums
-constexpr int kOffMax = kOffRed + 2 * 8 * 16 * 4;  // [2][2][128] half-row maxima
-constexpr int kOffL = kOffMax + 2 * 2 * 128 * 4;   // [2][128] half-row normalisers
-constexpr int kOffBar = kOffL + 2 * 128 * 4;
-constexpr int kNumBars = 2 * kStages + 8 + kRecvSlots + 1;
+constexpr int kOffRed = kOffP + 2 * kPBytes;      // [2 groups][4 warps][32] p partial sums
+constexpr int kOffRef = kOffRed + 2 * 4 * 32 * 4;  // [2][128] per-row reference of a block
+constexpr int kOffFin = kOffRef + 2 * 128 * 4;     // [2 groups][2][128] final (l, reference)
+constexpr int kOffBar = kOffFin + 2 * 2 * 128 * 4;
+constexpr int kNumBars = 2 * kStages + 8 + kRecvSlots + 3;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kSmemBytes = kOffMisc + 64 + 1024;
 constexpr int kTmemCols = 512;
@@ -77,11 +76,10 @@ constexpr uint32_t kIdescQK = make_idesc(1, 1, false, false, 128, kBN);
 constexpr uint32_t kIdescPV = make_idesc(1, 1, false, true, 128, kDvCta);
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleLog2 = 8.0f;
-// named barriers of the 256 softmax threads
-constexpr int kBarRed = 1;  // p sweep partial sums
-constexpr int kBarXs = 2;   // outgoing partial S staged
-constexpr int kBarMax = 3;  // half-row maxima
-constexpr int kBarL = 4;    // half-row normalisers
+// named barriers: per softmax warpgroup (128 threads) + g, and one of all 256
+constexpr int kBarXs0 = 1;   // outgoing partial S staged
+constexpr int kBarRed0 = 3;  // p sweep partial sums
+constexpr int kBarFin = 5;   // final normaliser of both groups
 static_assert(kSmemBytes <= 232448, "shared memory");
 static_assert(kKvStage % 1024 == 0, "stage alignment (128B-swizzle atoms)");
 // A gather warp waits on a stage's barrier for the phase of its own previous block there; if
@@ -134,17 +132,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* sX = reinterpret_cast<float*>(smem + kOffX);
   uint8_t* sXs = smem + kOffXs;
   float* sRed = reinterpret_cast<float*>(smem + kOffRed);
-  float* sMax = reinterpret_cast<float*>(smem + kOffMax);
-  float* sL = reinterpret_cast<float*>(smem + kOffL);
+  float* sRef = reinterpret_cast<float*>(smem + kOffRef);
+  float* sFin = reinterpret_cast<float*>(smem + kOffFin);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
   uint64_t* kv_full = bars;                 // [kStages] expect_tx + the gathered bytes
   uint64_t* kv_empty = bars + kStages;      // [kStages] MMA commit
   uint64_t* s_full = bars + 2 * kStages;    // [2] MMA commit
-  uint64_t* s_empty = s_full + 2;           // [2] 256 softmax arrivals
-  uint64_t* p_full = s_full + 4;            // [2] 256 softmax arrivals
+  uint64_t* s_empty = s_full + 2;           // [2] 128 arrivals of the block's warpgroup
+  uint64_t* p_full = s_full + 4;            // [2] 128 arrivals of the block's warpgroup
   uint64_t* o_done = s_full + 6;            // [2] MMA commit (PV of blocks i, i % 2)
   uint64_t* x_full = s_full + 8;            // [kRecvSlots] own expect_tx + the peer's bytes
   uint64_t* q_ready = x_full + kRecvSlots;  // 256 softmax arrivals: Q is in tensor memory
+  uint64_t* ref_full = q_ready + 1;         // [2] 128 arrivals: a block's reference is published
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
   int* s_len = reinterpret_cast<int*>(smem + kOffMisc + 8);
@@ -169,8 +168,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_empty[i], kSoftmaxThreads);
-      mbar_init(&p_full[i], kSoftmaxThreads);
+      mbar_init(&s_empty[i], 128);
+      mbar_init(&p_full[i], 128);
+      mbar_init(&ref_full[i], 128);
       mbar_init(&o_done[i], 1);
     }
     for (int i = 0; i < kRecvSlots; ++i) mbar_init(&x_full[i], 1);
@@ -298,20 +298,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------------ softmax / epilogue
-    // Warpgroup wg owns S columns [16 wg, 16 wg + 16) of every block and O columns
-    // [128 wg, 128 wg + 128) of this CTA's value half; both hold the same per-row state.
+    // Warpgroup wg handles blocks q = wg, wg + 2, ... (thread = head row over all 32 columns),
+    // so two blocks are in flight.  Per block:
+    //   1. load the own partial S(q), stage it and bulk-copy it to the peer's receive slot;
+    //   2. add the peer's part: z = S * scale * log2(e), invalid slots -inf; row max bz;
+    //   3. the block's per-row reference r_q: take r_{q-1} from the other group (published in
+    //      shared memory with an mbarrier), keep it unless bz exceeds it by more than 2^8 (lazy
+    //      rescaling, so P <= 256), publish r_q - the only serial link between the groups;
+    //   4. if the reference moved, rescale O in tensor memory between PV(q-1) and PV(q);
+    //      P = 2^(z - r_q) -> bf16 -> the group's P buffer; l accumulates relative to r_q.
+    // Both CTAs of the pair see identical S and take identical decisions.
     const int wg = warp >> 2;
     const int wq = warp & 3;
     const int h = (wq << 5) + lane;  // head row = TMEM lane (warp w owns lanes 32(w%4)..)
+    const int wtid = threadIdx.x & 127;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t tm = tmem_base + lane_off;
-    const int col0 = wg * kHalf;
-    const uint32_t o_cols = static_cast<uint32_t>(wg * (kDvCta / 2));
     const uint32_t peer_recv = map_to_rank(smem_u32(sX), peer);
     const uint32_t peer_x_full = map_to_rank(smem_u32(x_full), peer);
     const uint32_t hsw = static_cast<uint32_t>(h & 7);
     const size_t orow = static_cast<size_t>(row) * p.H + h;
     const bool head_ok = h < p.H;
+    const int bar_xs = kBarXs0 + wg, bar_red = kBarRed0 + wg;
+    uint8_t* stg_row = sXs + wg * kXSlot + h * (kBN * 4);  // this group's staging slot, row h
     bool ok = true;
 
     if (total > 0) {
@@ -342,240 +351,220 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto mask_of = [&](int s) {
       return __ballot_sync(0xFFFFFFFFu, static_cast<unsigned>(s) < static_cast<unsigned>(p.Lk));
     };
-    // validity masks of blocks q and q+1, and the pending slot load of block q+2
-    uint32_t m_cur = 0, m_nxt = 0;
-    int s_pf = -1;
-    if (total > 0) m_cur = mask_of(block_slot(idx_row, e0, len, 0, lane));
-    if (total > 1) m_nxt = mask_of(block_slot(idx_row, e0, len, blk_of(1), lane));
-    if (total > 2) s_pf = block_slot(idx_row, e0, len, blk_of(2), lane);
 
-    // Load this CTA's partial S(j) (this warpgroup's 16 columns) from tensor memory, stage it in
-    // shared memory and ship the whole 128 x 32 partial to the peer's receive slot
-    // j % kRecvSlots with one bulk copy.  Remote stores from the threads were measured slower:
-    // 16 KB of 16-byte st.async per block takes about 1000 cycles to issue.  Row h takes 128 B,
-    // 16-byte chunk c kept at chunk c ^ (h % 8) so that a warp's accesses spread over all banks.
-    //   Receive slots: four make reuse safe without a back-signal.  This CTA sends block j+1 only
-    //   after it received the peer's block j-1, which the peer sends only after it finished
-    //   reading the slot of block j-3 = (j+1) - 4.
-    //   Staging slots: j % 2.  Before the barrier of block j, thread 0 waits until its copies of
-    //   blocks <= j-1 have read their source, so slot (j+1) % 2 is free once all have passed it.
-    auto load_and_send = [&](int j, uint32_t (&dst)[kHalf]) {
-      if (ok && !mbar_wait(&s_full[j & 1], (j >> 1) & 1, abort_flag, 63)) ok = false;
+    // Steps 1-2 for block q: z[] = the full S(q) (unscaled), -inf at invalid slots.
+    // Staging: one slot per group, reused every other block; the group's leader waits until its
+    // previous copy has read the slot, and a barrier publishes that before anyone rewrites it.
+    // Receive slots q % 4: four make reuse safe without a back-signal.  This group sends block
+    // q+4 only after it received the peer group's block q+2, which that group sends only after
+    // it finished reading the slot of block q.
+    auto full_s = [&](int q, uint32_t vm, float (&z)[32]) {
+      if (wtid == 0) bulk_wait_read_all();
+      named_bar_sync(bar_xs, 128);
+      uint32_t v[32];
+      if (ok && !mbar_wait(&s_full[q & 1], (q >> 1) & 1, abort_flag, 63)) ok = false;
       ok = __all_sync(0xFFFFFFFFu, ok);  // tcgen05.ld is warp-collective
       if (ok) {
         tc_fence_after();
-        tmem_ld_32x32b_x16(tm + kTmemS + (j & 1) * kBN + col0, dst);
+        tmem_ld_32x32b_x32(tm + kTmemS + (q & 1) * kBN, v);
         tmem_ld_wait();
         tc_fence_before();
-        mbar_arrive(&s_empty[j & 1]);
-        uint8_t* stg = sXs + (j & 1) * kXSlot + h * (kBN * 4);
+        mbar_arrive(&s_empty[q & 1]);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const uint32_t c = static_cast<uint32_t>(4 * wg + i);
-          *reinterpret_cast<uint4*>(stg + ((c ^ hsw) << 4)) =
-              make_uint4(dst[4 * i], dst[4 * i + 1], dst[4 * i + 2], dst[4 * i + 3]);
-        }
+        for (int i = 0; i < 8; ++i)
+          *reinterpret_cast<uint4*>(stg_row + ((static_cast<uint32_t>(i) ^ hsw) << 4)) =
+              make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
         fence_proxy_async_smem();  // the bulk copy reads through the async proxy
       } else {
 #pragma unroll
-        for (int c = 0; c < kHalf; ++c) dst[c] = 0u;
+        for (int c = 0; c < 32; ++c) v[c] = 0u;
       }
-      if (threadIdx.x == 0) bulk_wait_read_all();
-      named_bar_sync(kBarXs, kSoftmaxThreads);
-      if (threadIdx.x == 0 && ok) {
-        const int sl = j % kRecvSlots;
-        bulk_copy_to_peer(peer_recv + static_cast<uint32_t>(sl * kXSlot), smem_u32(sXs + (j & 1) * kXSlot),
-                          kXSlot, peer_x_full + sl * 8);
+      named_bar_sync(bar_xs, 128);
+      const int sl = q % kRecvSlots;
+      if (wtid == 0) {
+        if (ok)
+          bulk_copy_to_peer(peer_recv + static_cast<uint32_t>(sl * kXSlot), smem_u32(sXs + wg * kXSlot), kXSlot,
+                            peer_x_full + sl * 8);
         bulk_commit_group();
+        mbar_arrive_expect_tx(&x_full[sl], kXSlot);
+      }
+      if (ok && !mbar_wait_cluster(&x_full[sl], (q / kRecvSlots) & 1, abort_flag, 64)) ok = false;
+      ok = __all_sync(0xFFFFFFFFu, ok);
+      const uint8_t* mine = reinterpret_cast<const uint8_t*>(sX) + sl * kXSlot + h * (kBN * 4);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float4 u = ok ? *reinterpret_cast<const float4*>(mine + ((static_cast<uint32_t>(i) ^ hsw) << 4))
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float2 a0 = add2(make_float2(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1])), make_float2(u.x, u.y));
+        const float2 a1 = add2(make_float2(__uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3])), make_float2(u.z, u.w));
+        z[4 * i] = a0.x;
+        z[4 * i + 1] = a0.y;
+        z[4 * i + 2] = a1.x;
+        z[4 * i + 3] = a1.y;
+      }
+      if (vm != 0xFFFFFFFFu) {
+#pragma unroll
+        for (int c = 0; c < 32; ++c)
+          if (!((vm >> c) & 1u)) z[c] = -INFINITY;
       }
     };
 
-    float m_ref = -INFINITY;  // running reference max (log2 domain), identical in all copies
-    float l = 0.f;            // this warpgroup's part of the normaliser, relative to m_ref
+    const float sc = p.scale_log2;  // > 0, so max(t) * sc = max(t * sc)
+    float r = -INFINITY;  // reference of this group's previous block; l is relative to it
+    float l = 0.f;
     float lse2 = -INFINITY;
-    const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
-    uint32_t cur[kHalf], nxt[kHalf];
-    if (total > 0) load_and_send(0, cur);
-    for (int q = 0; q < total; ++q) {
-      if (q + 1 < total) load_and_send(q + 1, nxt);
-
-      // ---- y = (own part + the peer's part of S(q)) * scale * log2(e) - off, where off is the
-      // reference the block is measured against: the running max (main blocks; 0 before the
-      // first valid entry) or the final lse (p sweep).  Invalid slots get -inf.
-      const int sl = q % kRecvSlots;
-      if (threadIdx.x == 0) mbar_arrive_expect_tx(&x_full[sl], kXSlot);
-      if (ok && !mbar_wait_cluster(&x_full[sl], (q / kRecvSlots) & 1, abort_flag, 64)) ok = false;
-      ok = __all_sync(0xFFFFFFFFu, ok);
-      const uint32_t vm = (m_cur >> col0) & 0xFFFFu;  // the same in every warp of the group
-      const bool main_blk = q < nblk;
-      const float off = main_blk ? (m_ref == -INFINITY ? 0.f : m_ref) : lse2;
-      float y[kHalf];
-      {
-        const uint8_t* mine = reinterpret_cast<const uint8_t*>(sX) + sl * kXSlot + h * (kBN * 4);
-        const float2 o2 = make_float2(-off, -off);
+    bool fin = false;
+    // Final normaliser and O: both groups' l brought to the last block's reference, which is
+    // the largest (references never decrease); each group stores its 128 value columns.
+    auto finish = [&]() {
+      sFin[(wg * 2) * 128 + h] = l;
+      sFin[(wg * 2 + 1) * 128 + h] = r;
+      named_bar_sync(kBarFin, kSoftmaxThreads);
+      const float l0 = sFin[h], r0 = sFin[128 + h], l1 = sFin[256 + h], r1 = sFin[384 + h];
+      const float rf = fmaxf(r0, r1);
+      const float l_tot = (r0 == -INFINITY ? 0.f : l0 * ex2_approx(r0 - rf)) +
+                          (r1 == -INFINITY ? 0.f : l1 * ex2_approx(r1 - rf));
+      lse2 = l_tot > 0.f ? rf + log2f(l_tot) : -INFINITY;
+      if (nblk == 0) return;
+      const int ql = nblk - 1;
+      if (ok) {
+        const bool got = mbar_wait(&o_done[ql & 1], (ql >> 1) & 1, abort_flag, 67);
+        ok = __all_sync(0xFFFFFFFFu, got);
+      }
+      if (!ok) return;
+      tc_fence_after();
+      const float inv_l = l_tot > 0.f ? 1.f / l_tot : 0.f;
+      const uint32_t o_cols = static_cast<uint32_t>(wg * (kDvCta / 2));
+#pragma unroll 1
+      for (int c0 = 0; c0 < kDvCta / 2; c0 += 16) {
+        uint32_t o[16];
+        tmem_ld_32x32b_x16(tm + kTmemO + o_cols + c0, o);
+        tmem_ld_wait();
+        if (!head_ok) continue;
+        const int col = static_cast<int>(rank) * kDvCta + static_cast<int>(o_cols) + c0;
+        if (p.n_split == 1) {
+          uint4 w0, w1;
+          w0.x = pack_bf16x2(__uint_as_float(o[0]) * inv_l, __uint_as_float(o[1]) * inv_l);
+          w0.y = pack_bf16x2(__uint_as_float(o[2]) * inv_l, __uint_as_float(o[3]) * inv_l);
+          w0.z = pack_bf16x2(__uint_as_float(o[4]) * inv_l, __uint_as_float(o[5]) * inv_l);
+          w0.w = pack_bf16x2(__uint_as_float(o[6]) * inv_l, __uint_as_float(o[7]) * inv_l);
+          w1.x = pack_bf16x2(__uint_as_float(o[8]) * inv_l, __uint_as_float(o[9]) * inv_l);
+          w1.y = pack_bf16x2(__uint_as_float(o[10]) * inv_l, __uint_as_float(o[11]) * inv_l);
+          w1.z = pack_bf16x2(__uint_as_float(o[12]) * inv_l, __uint_as_float(o[13]) * inv_l);
+          w1.w = pack_bf16x2(__uint_as_float(o[14]) * inv_l, __uint_as_float(o[15]) * inv_l);
+          uint4* dst = reinterpret_cast<uint4*>(p.out + orow * kDV + col);
+          dst[0] = w0;
+          dst[1] = w1;
+        } else {
+          float4* dst = reinterpret_cast<float4*>(p.part_o + (static_cast<size_t>(split) * p.B * p.Lq * p.H + orow) * kDV + col);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const uint32_t c = static_cast<uint32_t>(4 * wg + i);
-          const float4 u = ok ? *reinterpret_cast<const float4*>(mine + ((c ^ hsw) << 4))
-                              : make_float4(0.f, 0.f, 0.f, 0.f);
-          float2 a0 = add2(make_float2(__uint_as_float(cur[4 * i]), __uint_as_float(cur[4 * i + 1])),
-                           make_float2(u.x, u.y));
-          float2 a1 = add2(make_float2(__uint_as_float(cur[4 * i + 2]), __uint_as_float(cur[4 * i + 3])),
-                           make_float2(u.z, u.w));
-          a0 = fma2(a0, sc2, o2);
-          a1 = fma2(a1, sc2, o2);
-          y[4 * i] = a0.x;
-          y[4 * i + 1] = a0.y;
-          y[4 * i + 2] = a1.x;
-          y[4 * i + 3] = a1.y;
-        }
-        if (vm != 0xFFFFu) {
-#pragma unroll
-          for (int c = 0; c < kHalf; ++c)
-            if (!((vm >> c) & 1u)) y[c] = -INFINITY;
+          for (int c = 0; c < 16; c += 4)
+            dst[c / 4] = make_float4(__uint_as_float(o[c]) * inv_l, __uint_as_float(o[c + 1]) * inv_l,
+                                     __uint_as_float(o[c + 2]) * inv_l, __uint_as_float(o[c + 3]) * inv_l);
         }
       }
-      // advance the mask pipeline (the load of block q+2 was issued one iteration ago)
-      m_cur = m_nxt;
-      m_nxt = mask_of(s_pf);
-      s_pf = (q + 3 < total) ? block_slot(idx_row, e0, len, blk_of(q + 3), lane) : -1;
+      if (head_ok && rank == 0 && wg == 0) {
+        const float lse_nat = lse2 * kLn2;
+        if (p.n_split == 1) {
+          if (p.lse) p.lse[orow] = lse_nat;
+        } else {
+          p.part_lse[static_cast<size_t>(split) * p.B * p.Lq * p.H + orow] = lse_nat;
+        }
+      }
+    };
 
-      if (main_blk) {
-        // ---- online softmax of block q; y is measured against m_ref
-        float t8[8];
+    // mask of this group's next block and the pending slot load of the one after
+    uint32_t m_cur = mask_of((wg < total) ? block_slot(idx_row, e0, len, blk_of(wg), lane) : -1);
+    int s_pf = (wg + 2 < total) ? block_slot(idx_row, e0, len, blk_of(wg + 2), lane) : -1;
+    for (int q = wg; q < total; q += 2) {
+      const uint32_t vm = m_cur;
+      m_cur = mask_of(s_pf);
+      s_pf = (q + 4 < total) ? block_slot(idx_row, e0, len, blk_of(q + 4), lane) : -1;
+      if (q >= nblk && !fin) {
+        finish();
+        fin = true;
+      }
+      float t[32];
+      full_s(q, vm, t);
+      if (q < nblk) {
+        // ---- step 3: the block's reference
+        float m8[8];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) t8[c] = fmaxf(y[c], y[c + 8]);
-#pragma unroll
-        for (int c = 0; c < 4; ++c) t8[c] = fmaxf(t8[c], t8[c + 4]);
-        float by = fmaxf(fmaxf(t8[0], t8[2]), fmaxf(t8[1], t8[3]));
-        float* mx = sMax + (q & 1) * 256;  // double-buffered by block parity
-        mx[wg * 128 + h] = by;
-        named_bar_sync(kBarMax, kSoftmaxThreads);
-        by = fmaxf(by, mx[(wg ^ 1) * 128 + h]);
+        for (int c = 0; c < 8; ++c) m8[c] = fmaxf(fmaxf(t[c], t[c + 8]), fmaxf(t[c + 16], t[c + 24]));
+        const float bz = fmaxf(fmaxf(fmaxf(m8[0], m8[4]), fmaxf(m8[1], m8[5])),
+                               fmaxf(fmaxf(m8[2], m8[6]), fmaxf(m8[3], m8[7]))) * sc;
+        float rp = -INFINITY;
+        if (q > 0) {
+          if (ok && !mbar_wait(&ref_full[(q - 1) & 1], ((q - 1) >> 1) & 1, abort_flag, 68)) ok = false;
+          ok = __all_sync(0xFFFFFFFFu, ok);
+          rp = sRef[((q - 1) & 1) * 128 + h];
+        }
+        const float rq = (rp == -INFINITY) ? bz : ((bz > rp + kRescaleLog2) ? bz : rp);
+        sRef[(q & 1) * 128 + h] = rq;
+        mbar_arrive(&ref_full[q & 1]);
+        // ---- step 4: rescale O if the reference moved, then P
         const int pb = q & 1;
         if (ok && q >= 2) {  // P buffer pb was last read by PV(q-2)
           const bool got = mbar_wait(&o_done[pb], ((q - 2) >> 1) & 1, abort_flag, 65);
           ok = __all_sync(0xFFFFFFFFu, got);
         }
-        // Lazy rescale: the reference only moves (by the block's excess d) on the first valid
-        // entry or when a block exceeds it by more than 2^8, so P <= 256 stays well inside bf16
-        // range.  O is rescaled in tensor memory once PV(q-1) has landed (tcgen05.ld/st are
-        // warp-collective, so the whole warp walks its rows); each warpgroup its 128 columns.
-        const bool first = (m_ref == -INFINITY);
-        const bool move = first ? (by > -INFINITY) : (by > kRescaleLog2);
-        const float d = move ? by : 0.f;
-        if (ok) {
-          const bool scale_o = move && !first;
-          const float f = scale_o ? ex2_approx(-by) : 1.f;
-          if (__any_sync(0xFFFFFFFFu, scale_o)) {
-            const bool got = mbar_wait(&o_done[(q - 1) & 1], ((q - 1) >> 1) & 1, abort_flag, 66);
-            ok = __all_sync(0xFFFFFFFFu, got);
-            if (ok) {
-              tc_fence_after();
+        const bool moved = (rp != -INFINITY) && (rq != rp);
+        if (ok && __any_sync(0xFFFFFFFFu, moved)) {
+          const bool got = mbar_wait(&o_done[(q - 1) & 1], ((q - 1) >> 1) & 1, abort_flag, 66);
+          ok = __all_sync(0xFFFFFFFFu, got);
+          if (ok) {
+            const float f = moved ? ex2_approx(rp - rq) : 1.f;
+            tc_fence_after();
 #pragma unroll 1
-              for (int c0 = 0; c0 < kDvCta / 2; c0 += 16) {
-                uint32_t o[16];
-                tmem_ld_32x32b_x16(tm + kTmemO + o_cols + c0, o);
-                tmem_ld_wait();
+            for (int c0 = 0; c0 < kDvCta; c0 += 16) {
+              uint32_t o[16];
+              tmem_ld_32x32b_x16(tm + kTmemO + c0, o);
+              tmem_ld_wait();
 #pragma unroll
-                for (int c = 0; c < 16; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * f);
-                tmem_st_32x32b_x16(tm + kTmemO + o_cols + c0, o);
-              }
-              tmem_st_wait();
+              for (int c = 0; c < 16; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * f);
+              tmem_st_32x32b_x16(tm + kTmemO + c0, o);
             }
+            tmem_st_wait();
           }
-          l *= f;
-          if (move) m_ref = first ? by : m_ref + by;
         }
+        if (r != -INFINITY && r != rq) l *= ex2_approx(r - rq);
+        r = rq;
         if (ok) {
-          if (__any_sync(0xFFFFFFFFu, move)) {
-#pragma unroll
-            for (int c = 0; c < kHalf; ++c) y[c] -= d;
-          }
-          uint32_t pk[kHalf / 2];
+          const bool live = rq != -INFINITY;
+          const float2 nr2 = make_float2(-rq, -rq), sc2 = make_float2(sc, sc);
+          uint32_t pk[16];
           float2 rs[4];
 #pragma unroll
-          for (int c = 0; c < kHalf; c += 2) {
-            const float2 pp = make_float2(ex2_approx(y[c]), ex2_approx(y[c + 1]));
+          for (int c = 0; c < 32; c += 2) {
+            const float2 y2 = fma2(make_float2(t[c], t[c + 1]), sc2, nr2);
+            const float2 pp = live ? make_float2(ex2_approx(y2.x), ex2_approx(y2.y)) : make_float2(0.f, 0.f);
             rs[(c >> 1) & 3] = (c < 8) ? pp : add2(rs[(c >> 1) & 3], pp);
             pk[c >> 1] = pack_bf16x2(pp.x, pp.y);
           }
           const float2 r2 = add2(add2(rs[0], rs[1]), add2(rs[2], rs[3]));
           l += r2.x + r2.y;
-          uint8_t* pbuf = sP + pb * kPBytes;  // row h: 64 B, 64B-swizzled; this half = chunks 2wg, 2wg+1
-          *reinterpret_cast<uint4*>(pbuf + swizzled_offset(h, 2 * wg, 64)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          *reinterpret_cast<uint4*>(pbuf + swizzled_offset(h, 2 * wg + 1, 64)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          uint8_t* pbuf = sP + pb * kPBytes;  // row h: 64 B, 64B-swizzled
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            *reinterpret_cast<uint4*>(pbuf + swizzled_offset(h, j, 64)) =
+                make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
           fence_proxy_async_smem();
           tc_fence_before();
           mbar_arrive(&p_full[pb]);
         }
-        if (q == nblk - 1) {
-          // ---- final O: total normaliser from both halves, wait for the last PV, store this
-          // warpgroup's 128 value columns
-          sL[wg * 128 + h] = l;
-          named_bar_sync(kBarL, kSoftmaxThreads);
-          const float l_tot = sL[h] + sL[128 + h];
-          if (ok) {
-            const bool got = mbar_wait(&o_done[pb], (q >> 1) & 1, abort_flag, 67);
-            ok = __all_sync(0xFFFFFFFFu, got);
-          }
-          if (ok) {
-            tc_fence_after();
-            const float inv_l = l_tot > 0.f ? 1.f / l_tot : 0.f;
-            lse2 = l_tot > 0.f ? m_ref + log2f(l_tot) : -INFINITY;
-#pragma unroll 1
-            for (int c0 = 0; c0 < kDvCta / 2; c0 += 16) {
-              uint32_t o[16];
-              tmem_ld_32x32b_x16(tm + kTmemO + o_cols + c0, o);
-              tmem_ld_wait();
-              if (!head_ok) continue;
-              const int col = static_cast<int>(rank) * kDvCta + static_cast<int>(o_cols) + c0;
-              if (p.n_split == 1) {
-                uint4 w0, w1;
-                w0.x = pack_bf16x2(__uint_as_float(o[0]) * inv_l, __uint_as_float(o[1]) * inv_l);
-                w0.y = pack_bf16x2(__uint_as_float(o[2]) * inv_l, __uint_as_float(o[3]) * inv_l);
-                w0.z = pack_bf16x2(__uint_as_float(o[4]) * inv_l, __uint_as_float(o[5]) * inv_l);
-                w0.w = pack_bf16x2(__uint_as_float(o[6]) * inv_l, __uint_as_float(o[7]) * inv_l);
-                w1.x = pack_bf16x2(__uint_as_float(o[8]) * inv_l, __uint_as_float(o[9]) * inv_l);
-                w1.y = pack_bf16x2(__uint_as_float(o[10]) * inv_l, __uint_as_float(o[11]) * inv_l);
-                w1.z = pack_bf16x2(__uint_as_float(o[12]) * inv_l, __uint_as_float(o[13]) * inv_l);
-                w1.w = pack_bf16x2(__uint_as_float(o[14]) * inv_l, __uint_as_float(o[15]) * inv_l);
-                uint4* dst = reinterpret_cast<uint4*>(p.out + orow * kDV + col);
-                dst[0] = w0;
-                dst[1] = w1;
-              } else {
-                float4* dst = reinterpret_cast<float4*>(
-                    p.part_o + (static_cast<size_t>(split) * p.B * p.Lq * p.H + orow) * kDV + col);
-#pragma unroll
-                for (int c = 0; c < 16; c += 4)
-                  dst[c / 4] = make_float4(__uint_as_float(o[c]) * inv_l, __uint_as_float(o[c + 1]) * inv_l,
-                                           __uint_as_float(o[c + 2]) * inv_l, __uint_as_float(o[c + 3]) * inv_l);
-              }
-            }
-            if (head_ok && rank == 0 && wg == 0) {
-              const float lse_nat = lse2 * kLn2;
-              if (p.n_split == 1) {
-                if (p.lse) p.lse[orow] = lse_nat;
-              } else {
-                p.part_lse[static_cast<size_t>(split) * p.B * p.Lq * p.H + orow] = lse_nat;
-              }
-            }
-          }
-        }
       } else {
-        // ---- p sweep: P = exp2(y) (y measured against lse) summed over heads h < H, / H.  Blocks
-        // alternate between the two CTAs (both computed the same S); each warpgroup sums its 16
-        // columns.
+        // ---- p sweep: P = 2^(t * sc - lse2) summed over heads h < H, divided by H.  Blocks
+        // alternate between the two CTAs (both computed the same S).
         const int blk = blk_of(q);
         if ((blk & 1) == static_cast<int>(rank)) {
           const bool live = ok && head_ok && lse2 != -INFINITY;
-          float v[kHalf];
+          float v[32];
 #pragma unroll
-          for (int c = 0; c < kHalf; ++c) v[c] = live ? ex2_approx(y[c]) : 0.f;
-          // butterfly reduce-scatter: lane L ends with column L % 16 summed over its 16-lane
-          // half, then over the whole warp
+          for (int c = 0; c < 32; ++c) v[c] = live ? ex2_approx(fmaf(t[c], sc, -lse2)) : 0.f;
+          // butterfly reduce-scatter over the warp: lane L ends with column L summed over the
+          // warp's 32 heads
 #pragma unroll
-          for (int off2 = 8; off2 >= 1; off2 >>= 1) {
+          for (int off2 = 16; off2 >= 1; off2 >>= 1) {
             const bool upper = (lane & off2) != 0;
 #pragma unroll
             for (int i = 0; i < off2; ++i) {
@@ -584,22 +573,18 @@ __global__ void __launch_bounds__(kThreads, 1)
               v[i] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, off2);
             }
           }
-          v[0] += __shfl_xor_sync(0xFFFFFFFFu, v[0], 16);
-          float* red = sRed + ((blk >> 1) & 1) * 128;  // double-buffered by own-block parity
-          if (lane < 16) red[warp * 16 + lane] = v[0];
-          named_bar_sync(kBarRed, kSoftmaxThreads);
-          if (wq == 0 && lane < 16 && ok) {
-            const float* r4 = red + wg * 64;  // warps 4wg .. 4wg+3
-            const float tot = r4[lane] + r4[16 + lane] + r4[32 + lane] + r4[48 + lane];
-            const int slot2 = e0 + blk * kBN + col0 + lane;
-            if (slot2 < e1)
-              p.p_sel[static_cast<size_t>(row) * p.k + slot2] = ((vm >> lane) & 1u) ? tot / p.H : 0.f;
+          float* red = sRed + wg * 128;
+          red[wq * 32 + lane] = v[0];
+          named_bar_sync(bar_red, 128);
+          if (wq == 0 && ok) {
+            const float tot = red[lane] + red[32 + lane] + red[64 + lane] + red[96 + lane];
+            const int slot2 = e0 + blk * kBN + lane;
+            if (slot2 < e1) p.p_sel[static_cast<size_t>(row) * p.k + slot2] = ((vm >> lane) & 1u) ? tot / p.H : 0.f;
           }
         }
       }
-#pragma unroll
-      for (int c = 0; c < kHalf; ++c) cur[c] = nxt[c];
     }
+    if (!fin) finish();
 
     // p emission: slots past the effective length are empty (p = 0)
     if (p.p_sel != nullptr && rank == 0) {
@@ -607,6 +592,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         p.p_sel[static_cast<size_t>(row) * p.k + x2] = 0.f;
     }
     if (nblk == 0 && head_ok) {  // no valid entry in this split
+      const uint32_t o_cols = static_cast<uint32_t>(wg * (kDvCta / 2));
       for (int c = 0; c < kDvCta / 2; ++c) {
         const int col = static_cast<int>(rank) * kDvCta + static_cast<int>(o_cols) + c;
         if (p.n_split == 1)
