@@ -124,7 +124,8 @@ dsa_status launch_indexer(const void* q, const void* kk, const float* w, float* 
   if (base >= 2L * sms) {
     p.kc = p.n_kt;
   } else {
-    const long splits = (4L * sms + base - 1) / base;
+    // about 16 items per CTA, so that whole items left over at the end cost little
+    const long splits = (16L * sms + base - 1) / base;
     p.kc = static_cast<int>(std::max<long>(4, (p.n_kt + splits - 1) / splits));
   }
   p.kc = std::min(p.kc, p.n_kt);
@@ -279,7 +280,8 @@ dsa_status launch_mla(const void* q, const void* kv, const int32_t* idx, int B, 
   }
   if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
   if (sp.n_split > 1) {
-    dsa::mla::combine_kernel<D_V><<<rows * H, 128, 0, stream>>>(
+    const int cgrid = (rows * H + dsa::mla::kCombineWarps - 1) / dsa::mla::kCombineWarps;
+    dsa::mla::combine_kernel<D_V><<<cgrid, dsa::mla::kCombineWarps * 32, 0, stream>>>(
         p.part_o, p.part_lse, sp.n_split, rows * H, static_cast<__nv_bfloat16*>(out), lse);
     return launch_result();
   }

@@ -7,7 +7,8 @@
 // registers without any cross-lane reduction; only the [Lq, Lk] scores reach HBM.
 //
 // Persistent, warp-specialised CTA (one per SM):
-//   warp 0        TMA producer: the q_I group once per work item, then k_I tiles (6 stages)
+//   warp 0        TMA producer: the q_I group once per work item, then k_I tiles (12 stages
+//                 for decode, 6 otherwise)
 //   warp 1        MMA issuer (one thread): d_I/32 MMAs of 128 x N x 32 per tile
 //   warp 2        TMEM allocator (2 accumulators of N columns, double-buffered)
 //   warps 4..11   epilogue: tcgen05.ld -> ReLU * w -> head sum -> mask -> store
@@ -24,7 +25,6 @@ namespace indexer {
 
 constexpr int kEpiWarps = 8;
 constexpr int kThreads = 128 + kEpiWarps * 32;
-constexpr int kStages = 6;
 constexpr int kTileKeys = 128;
 
 struct Params {
@@ -40,6 +40,9 @@ struct Params {
 
 template <int H_I, int D_I, int G>
 struct Cfg {
+  // k_I ring depth: decode streams k_I from HBM with little else per tile, so it keeps twice
+  // as many tiles in flight
+  static constexpr int kStages = (G == 1) ? 12 : 6;
   static constexpr int N = G * H_I;                      // MMA N (columns per accumulator)
   static constexpr int kQBytes = N * D_I;                // q_I group tile
   static constexpr int kKBytes = kTileKeys * D_I;        // k_I tile
@@ -102,8 +105,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* sW = reinterpret_cast<float*>(smem + C::kOffW);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
   uint64_t* k_full = bars;
-  uint64_t* k_empty = bars + kStages;
-  uint64_t* q_full = bars + 2 * kStages;
+  uint64_t* k_empty = bars + C::kStages;
+  uint64_t* q_full = bars + 2 * C::kStages;
   uint64_t* q_empty = q_full + 2;
   uint64_t* acc_full = q_full + 4;
   uint64_t* acc_empty = q_full + 6;
@@ -114,7 +117,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&k_full[s], 1);
       mbar_init(&k_empty[s], 1);
     }
@@ -158,7 +161,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_expect_tx(&k_full[ks], C::kKBytes);
           tma_load_2d(sK + ks * C::kKBytes, &tm_k, &k_full[ks], 0,
                       b * p.Lk + (kt0 + tt) * kTileKeys);
-          if (++ks == kStages) {
+          if (++ks == C::kStages) {
             ks = 0;
             kph ^= 1;
           }
@@ -197,7 +200,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           mma_commit(&k_empty[ks]);
           mma_commit(&acc_full[ab]);
-          if (++ks == kStages) {
+          if (++ks == C::kStages) {
             ks = 0;
             kph ^= 1;
           }
@@ -214,10 +217,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int wg = e >> 7;            // warpgroup 0 / 1
     const int sp = warp & 3;          // TMEM sub-partition this warp may access
     const int row = sp * 32 + lane;   // accumulator row = key within the tile
-    const bool worker = C::kSplitWG || wg == 0;
+    // G >= 2: both groups take every tile (half of the queries each).  G == 1: the groups take
+    // turns by tile, each owning one of the two accumulator buffers.
     bool ok = true;
-    int ab = 0;
-    uint32_t aph = 0;
+    int gt = 0;  // tiles with an MMA seen so far, over all items (both groups count every one)
     int it = 0;
     for (int u = blockIdx.x; u < p.n_items; u += gridDim.x, ++it) {
       int b, qg, kc, kt0, kt1, n_comp;
@@ -231,8 +234,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       named_bar_sync(1, 256);
       const size_t row_base = static_cast<size_t>(b) * p.Lq;
-      for (int tt = 0; tt < n_comp; ++tt) {
-        if (!worker || !ok) continue;
+      for (int tt = 0; tt < n_comp; ++tt, ++gt) {
+        const int ab = gt & 1;
+        const uint32_t aph = (gt >> 1) & 1;
+        if (!(C::kSplitWG || ab == wg) || !ok) continue;
         const bool got = mbar_wait(&acc_full[ab], aph, abort_flag, 6);
         if (!__all_sync(0xFFFFFFFFu, got)) {  // tcgen05.ld below is warp-collective
           ok = false;  // keep reaching the named barriers; skip the remaining work
@@ -242,7 +247,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float acc[C::kQPerWG];
 #pragma unroll
         for (int g = 0; g < C::kQPerWG; ++g) acc[g] = 0.f;
-        const int col0 = wg * C::kColsPerWG;  // 0 when not split
+        const int col0 = C::kSplitWG ? wg * C::kColsPerWG : 0;
         const uint32_t taddr = tmem_base + (static_cast<uint32_t>(sp * 32) << 16) + ab * C::N + col0;
 #pragma unroll
         for (int ch = 0; ch < C::kColsPerWG / 32; ++ch) {
@@ -257,8 +262,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_before();
         mbar_arrive(&acc_empty[ab]);
-        ab ^= 1;
-        if (ab == 0) aph ^= 1;
         const int s = (kt0 + tt) * kTileKeys + row;
         if (s < p.Lk) {
 #pragma unroll
@@ -269,13 +272,6 @@ __global__ void __launch_bounds__(kThreads, 1)
               p.scores[(row_base + i) * p.Lk + s] = (s <= t) ? acc[g] : -INFINITY;
             }
           }
-        }
-      }
-      // keep the accumulator ring in step on the idle warpgroup
-      if (!worker) {
-        for (int tt = 0; tt < n_comp; ++tt) {
-          ab ^= 1;
-          if (ab == 0) aph ^= 1;
         }
       }
       // fully masked tiles: no MMA, just -inf

@@ -437,29 +437,56 @@ done:
 }
 
 // Split-KV combine: out = sum_s exp(lse_s - lse) * O_s,  lse = ln sum_s exp(lse_s).
+// Split-KV combine: out[rh, :] = sum_s w_s * part_o[s, rh, :] with w_s = exp(lse_s - lse_all),
+// lse_all = log sum_s exp(lse_s).  One warp per (row, head): the splits' lse values are
+// reduced with shuffles and every lane streams D_V / 32 contiguous columns of each split, so a
+// warp issues all of its loads at once.
+constexpr int kCombineWarps = 8;
+
 template <int D_V>
-__global__ void combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_lse,
-                               int n_split, int rows_h, __nv_bfloat16* __restrict__ out, float* lse) {
-  const int rh = blockIdx.x;  // (row, head)
-  if (rh >= rows_h) return;
+__global__ void __launch_bounds__(kCombineWarps * 32)
+    combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_lse, int n_split,
+                   int rows_h, __nv_bfloat16* __restrict__ out, float* lse) {
+  constexpr int kPer = D_V / 32;  // columns per lane
+  static_assert(kPer % 2 == 0, "D_V");
+  const int rh = blockIdx.x * kCombineWarps + static_cast<int>(threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (rh >= rows_h) return;  // warp-uniform
   float m = -INFINITY;
-  for (int s = 0; s < n_split; ++s) m = fmaxf(m, part_lse[static_cast<size_t>(s) * rows_h + rh]);
+  for (int s = lane; s < n_split; s += 32) m = fmaxf(m, part_lse[static_cast<size_t>(s) * rows_h + rh]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
   float denom = 0.f;
-  for (int s = 0; s < n_split; ++s) {
+  for (int s = lane; s < n_split; s += 32) {
     const float ls = part_lse[static_cast<size_t>(s) * rows_h + rh];
     denom += (ls == -INFINITY) ? 0.f : expf(ls - m);
   }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) denom += __shfl_xor_sync(0xFFFFFFFFu, denom, o);
   const float lse_all = (denom > 0.f) ? m + logf(denom) : -INFINITY;
-  for (int c = threadIdx.x; c < D_V; c += blockDim.x) {
-    float acc = 0.f;
-    for (int s = 0; s < n_split; ++s) {
-      const float ls = part_lse[static_cast<size_t>(s) * rows_h + rh];
-      if (ls == -INFINITY) continue;
-      acc += expf(ls - lse_all) * part_o[(static_cast<size_t>(s) * rows_h + rh) * D_V + c];
+  float acc[kPer];
+#pragma unroll
+  for (int c = 0; c < kPer; ++c) acc[c] = 0.f;
+#pragma unroll 2
+  for (int s = 0; s < n_split; ++s) {
+    const float ls = part_lse[static_cast<size_t>(s) * rows_h + rh];
+    if (ls == -INFINITY) continue;  // warp-uniform
+    const float w = expf(ls - lse_all);
+    const float* src = part_o + (static_cast<size_t>(s) * rows_h + rh) * D_V + lane * kPer;
+#pragma unroll
+    for (int c = 0; c < kPer; c += 2) {
+      const float2 v = *reinterpret_cast<const float2*>(src + c);
+      acc[c] = fmaf(w, v.x, acc[c]);
+      acc[c + 1] = fmaf(w, v.y, acc[c + 1]);
     }
-    out[static_cast<size_t>(rh) * D_V + c] = __float2bfloat16_rn(acc);
   }
-  if (threadIdx.x == 0 && lse != nullptr) lse[rh] = lse_all;
+  __nv_bfloat16* dst = out + static_cast<size_t>(rh) * D_V + lane * kPer;
+#pragma unroll
+  for (int c = 0; c < kPer; c += 2) {
+    const __nv_bfloat162 pr = __floats2bfloat162_rn(acc[c], acc[c + 1]);
+    *reinterpret_cast<__nv_bfloat162*>(dst + c) = pr;
+  }
+  if (lane == 0 && lse != nullptr) lse[rh] = lse_all;
 }
 
 }  // namespace mla

@@ -327,20 +327,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       // This CTA's 288 dims of Q into tensor memory: dims [8j, 8j+8) of the slice -> columns
       // [4j, 4j+4), in 9 groups of 16 columns (warpgroup 0 takes groups 0-4, 1 takes 5-8).
       // Heads >= H get zeros.
+      // All of a thread's loads are issued before the first store, so the prologue costs one
+      // memory round trip rather than five.
       const __nv_bfloat16* qrow = p.q + orow * kDQK;
-#pragma unroll 1
-      for (int grp = wg * 5; grp < (wg == 0 ? 5 : 9); ++grp) {
-        uint4 v[4];
+      const int g0 = wg * 5, ng = wg == 0 ? 5 : 4;
+      uint4 v[20];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int j = grp * 4 + i;
-          const int d = j < 32 ? static_cast<int>(rank) * kDvCta + j * 8
-                               : kDV + static_cast<int>(rank) * kRopeCta + (j - 32) * 8;
-          v[i] = head_ok ? __ldg(reinterpret_cast<const uint4*>(qrow + d)) : make_uint4(0u, 0u, 0u, 0u);
+      for (int i = 0; i < 20; ++i) {
+        const int j = g0 * 4 + i;
+        const int d = j < 32 ? static_cast<int>(rank) * kDvCta + j * 8
+                             : kDV + static_cast<int>(rank) * kRopeCta + (j - 32) * 8;
+        v[i] = (head_ok && i < ng * 4) ? __ldg(reinterpret_cast<const uint4*>(qrow + d)) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int gi = 0; gi < 5; ++gi) {
+        if (gi < ng) {
+          const uint32_t r[16] = {v[4 * gi].x,     v[4 * gi].y,     v[4 * gi].z,     v[4 * gi].w,
+                                  v[4 * gi + 1].x, v[4 * gi + 1].y, v[4 * gi + 1].z, v[4 * gi + 1].w,
+                                  v[4 * gi + 2].x, v[4 * gi + 2].y, v[4 * gi + 2].z, v[4 * gi + 2].w,
+                                  v[4 * gi + 3].x, v[4 * gi + 3].y, v[4 * gi + 3].z, v[4 * gi + 3].w};
+          tmem_st_32x32b_x16(tm + kTmemQ + (g0 + gi) * 16, r);
         }
-        const uint32_t r[16] = {v[0].x, v[0].y, v[0].z, v[0].w, v[1].x, v[1].y, v[1].z, v[1].w,
-                                v[2].x, v[2].y, v[2].z, v[2].w, v[3].x, v[3].y, v[3].z, v[3].w};
-        tmem_st_32x32b_x16(tm + kTmemQ + grp * 16, r);
       }
       tmem_st_wait();
       tc_fence_before();
