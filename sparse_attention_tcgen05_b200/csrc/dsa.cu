@@ -241,7 +241,9 @@ dsa_status launch_mla(const void* q, const void* kv, const int32_t* idx, int B, 
   const long grid = static_cast<long>(rows) * Cfg::kNdv * sp.n_split;
   if (grid > INT32_MAX) return DSA_ERR_UNSUPPORTED;
   if constexpr (D_QK == dsa::mla_pair::kDQK && D_V == dsa::mla_pair::kDV) {
-    // cluster of two CTAs per (row, split): QK dims and value dims split between them
+    // cluster of two CTAs per (row, split): QK dims and value dims split between them; with two
+    // splits, both pairs of a row form one cluster of four that combines in the kernel
+    p.fuse2 = (sp.n_split == 2) ? 1 : 0;
     // kv as [B * Lk rows, 576 dims]: one-row boxes of 64 dims (SW128) and of the 32 rope dims
     // (SW64) for the row gathers
     CUtensorMap tm_main, tm_rope;
@@ -261,12 +263,13 @@ dsa_status launch_mla(const void* q, const void* kv, const int32_t* idx, int B, 
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.x = p.fuse2 ? 4 : 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     if (cudaLaunchKernelEx(&cfg, kern, tm_main, tm_rope, p) != cudaSuccess) return DSA_ERR_CUDA;
+    if (p.fuse2) return launch_result();
   } else {
     CUtensorMap tm_q;
     if (!encode_2d(&tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, D_QK, static_cast<uint64_t>(rows) * H,

@@ -39,14 +39,16 @@ struct Params {
   const __nv_bfloat16* q;  // [rows][H][d_qk] (read directly by the 576-d pair kernel)
   const __nv_bfloat16* kv;
   const int32_t* idx;
-  __nv_bfloat16* out;   // final output (n_split == 1)
-  float* lse;           // nullable (n_split == 1)
+  __nv_bfloat16* out;   // final output (n_split == 1, or fuse2)
+  float* lse;           // nullable (n_split == 1, or fuse2)
   float* p_sel;         // nullable
   float* part_o;        // [n_split][rows][H][d_v] fp32 (n_split > 1)
   float* part_lse;      // [n_split][rows][H]       fp32 (n_split > 1)
   int B, Lq, Lk, H, k;
   int n_split, per_split;  // entries of the idx row per split (multiple of kBN)
   float scale_log2;        // softmax scale * log2(e)
+  int fuse2;               // 576-d pair kernel, n_split == 2: both splits of a row form one
+                           // cluster of four and combine in the kernel (no combine launch)
 };
 
 template <int D_QK, int D_V>

@@ -150,8 +150,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const uint32_t rank = cluster_ctarank();
-  const uint32_t peer = rank ^ 1u;
+  const uint32_t crank = cluster_ctarank();
+  const uint32_t rank = crank & 1u;  // which half of the dims (within the pair)
+  const uint32_t peer = crank ^ 1u;  // cluster rank of the pair's other CTA
 
   const int pair = blockIdx.x >> 1;
   const int split = pair % p.n_split;
@@ -417,6 +418,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
 
     const float sc = p.scale_log2;  // > 0, so max(t) * sc = max(t * sc)
+    // Fused combine of two splits: this CTA finalises heads [64 split, 64 split + 64) and
+    // exports the other heads' normalised partial O and lse for the other split's CTA.
+    const bool own_head = (h >> 6) == split;
+    float own_inv_l = 0.f;
     float r = -INFINITY;  // reference of this group's previous block; l is relative to it
     float l = 0.f;
     float lse2 = -INFINITY;
@@ -441,7 +446,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) return;
       tc_fence_after();
       const float inv_l = l_tot > 0.f ? 1.f / l_tot : 0.f;
+      own_inv_l = inv_l;
       const uint32_t o_cols = static_cast<uint32_t>(wg * (kDvCta / 2));
+      if (p.fuse2 && own_head) return;  // finalised after the cluster barrier, from tensor memory
 #pragma unroll 1
       for (int c0 = 0; c0 < kDvCta / 2; c0 += 16) {
         uint32_t o[16];
@@ -449,7 +456,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld_wait();
         if (!head_ok) continue;
         const int col = static_cast<int>(rank) * kDvCta + static_cast<int>(o_cols) + c0;
-        if (p.n_split == 1) {
+        if (p.n_split == 1 && !p.fuse2) {
           uint4 w0, w1;
           w0.x = pack_bf16x2(__uint_as_float(o[0]) * inv_l, __uint_as_float(o[1]) * inv_l);
           w0.y = pack_bf16x2(__uint_as_float(o[2]) * inv_l, __uint_as_float(o[3]) * inv_l);
@@ -598,7 +605,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int x2 = e0 + nblk * kBN + static_cast<int>(threadIdx.x); x2 < e1; x2 += kSoftmaxThreads)
         p.p_sel[static_cast<size_t>(row) * p.k + x2] = 0.f;
     }
-    if (nblk == 0 && head_ok) {  // no valid entry in this split
+    if (nblk == 0 && head_ok && !(p.fuse2 && own_head)) {  // no valid entry in this split
       const uint32_t o_cols = static_cast<uint32_t>(wg * (kDvCta / 2));
       for (int c = 0; c < kDvCta / 2; ++c) {
         const int col = static_cast<int>(rank) * kDvCta + static_cast<int>(o_cols) + c;
@@ -615,8 +622,69 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
+    if (p.fuse2) {
+      // ---- combine with the other split: its exports are visible after the cluster barrier
+      // (release/acquire at cluster scope); every thread of all four CTAs takes it once here
+      // (the other roles at the end).  out = w_own * O_own + w_other * O_other, w = e^(lse - lse_all).
+      tc_fence_before();
+      __syncwarp();
+      cluster_barrier();
+      if (own_head) {  // warp-uniform (a warp covers 32 heads of one 64-head half)
+        const size_t rows_h = static_cast<size_t>(p.B) * p.Lq * p.H;
+        const float lse_o = head_ok ? p.part_lse[static_cast<size_t>(split ^ 1) * rows_h + orow] : -INFINITY;
+        const float lse_m = (ok && nblk > 0 && head_ok) ? lse2 * kLn2 : -INFINITY;  // natural log
+        const float mx = fmaxf(lse_m, lse_o);
+        const float em = lse_m == -INFINITY ? 0.f : expf(lse_m - mx);
+        const float eo = lse_o == -INFINITY ? 0.f : expf(lse_o - mx);
+        const float den = em + eo;
+        const float wm = den > 0.f ? em / den * own_inv_l : 0.f;  // own O is not yet normalised
+        const float wo = den > 0.f ? eo / den : 0.f;
+        const uint32_t o_cols = static_cast<uint32_t>(wg * (kDvCta / 2));
+        const float* other = p.part_o + (static_cast<size_t>(split ^ 1) * rows_h + orow) * kDV;
+        const bool need_tm = __any_sync(0xFFFFFFFFu, em > 0.f);  // tcgen05.ld is warp-collective
+        if (need_tm) tc_fence_after();
+#pragma unroll 1
+        for (int c0 = 0; c0 < kDvCta / 2; c0 += 16) {
+          uint32_t o[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c) o[c] = 0u;
+          if (need_tm) {
+            tmem_ld_32x32b_x16(tm + kTmemO + o_cols + c0, o);
+            tmem_ld_wait();
+          }
+          if (!head_ok) continue;
+          const int col = static_cast<int>(rank) * kDvCta + static_cast<int>(o_cols) + c0;
+          float r[16];
+#pragma unroll
+          for (int c = 0; c < 16; c += 4) {
+            const float4 u = wo > 0.f ? *reinterpret_cast<const float4*>(other + col + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+            r[c] = fmaf(wo, u.x, em > 0.f ? wm * __uint_as_float(o[c]) : 0.f);
+            r[c + 1] = fmaf(wo, u.y, em > 0.f ? wm * __uint_as_float(o[c + 1]) : 0.f);
+            r[c + 2] = fmaf(wo, u.z, em > 0.f ? wm * __uint_as_float(o[c + 2]) : 0.f);
+            r[c + 3] = fmaf(wo, u.w, em > 0.f ? wm * __uint_as_float(o[c + 3]) : 0.f);
+          }
+          uint4 w0, w1;
+          w0.x = pack_bf16x2(r[0], r[1]);
+          w0.y = pack_bf16x2(r[2], r[3]);
+          w0.z = pack_bf16x2(r[4], r[5]);
+          w0.w = pack_bf16x2(r[6], r[7]);
+          w1.x = pack_bf16x2(r[8], r[9]);
+          w1.y = pack_bf16x2(r[10], r[11]);
+          w1.z = pack_bf16x2(r[12], r[13]);
+          w1.w = pack_bf16x2(r[14], r[15]);
+          uint4* dst = reinterpret_cast<uint4*>(p.out + orow * kDV + col);
+          dst[0] = w0;
+          dst[1] = w1;
+        }
+        if (head_ok && rank == 0 && wg == 0 && p.lse) p.lse[orow] = den > 0.f ? mx + logf(den) : -INFINITY;
+      }
+    }
   }
 done:
+  if (p.fuse2 && warp >= kMmaWarp) {  // the softmax roles took this one above
+    __syncwarp();
+    cluster_barrier();
+  }
   tc_fence_before();
   __syncthreads();
   // neither CTA may leave while its peer can still store into its shared memory

@@ -155,6 +155,23 @@ def test_mla_full_dims_decode_split_and_p(dsa):
     _mla_case(dsa, wl, idx, emit_p=True)    # p emission keeps one CTA per value half
 
 
+def test_mla_decode_two_splits_combined_in_kernel(dsa):
+    # 32 decode rows -> two KV splits per row whose partial results are combined inside the
+    # attention kernel (the two pairs of a row form one cluster).  H = 100 leaves the last
+    # warp of heads partly empty; some rows have an empty first or second split.
+    wl = dsa_inputs.custom("mla_fuse2", 17, 32, 1, 3000, 64, 128, 16, 2048, 100, 576, 512,
+                           1 / math.sqrt(192))
+    rng = np.random.default_rng(21)
+    idx = np.stack([rng.permutation(3000)[:2048] for _ in range(32)]).astype(np.int32)
+    idx = idx.reshape(32, 1, 2048)
+    idx[0, 0, 600:] = -1        # second split empty
+    idx[1, 0, :1500] = -1       # first split empty
+    idx[2, 0, 1024:] = -1       # exactly the first split
+    idx[3, 0, 40:2000] = -1     # a few entries at both ends
+    idx[4, 0, :2047] = -1       # a single valid slot, in the second split
+    _mla_case(dsa, wl, idx)
+
+
 def test_mla_fewer_heads_and_short_sets(dsa):
     wl = dsa_inputs.custom("mla_h20", 13, 1, 6, 700, 64, 128, 16, 40, 20, 576, 512, 0.05)
     rng = np.random.default_rng(2)
