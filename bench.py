@@ -71,6 +71,36 @@ def algorithmic(wl):
     return {"indexer": ix, "topk": tk, "sparse_mla": ml, "indexer_kl": kl}
 
 
+def source_hash():
+    """Hash of the CUDA sources and the C header: DRAM traffic recorded under profiles/ is
+    reported only while the kernels it was measured on are unchanged."""
+    import hashlib
+
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "sparse_attention_tcgen05_b200", "csrc")
+    for name in sorted(os.listdir(csrc)) + ["../../include/dsa.h"]:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()[:12]
+
+
+def measured_traffic(workload, kernel):
+    """DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of `kernel` on
+    `workload` from profiles/dram_traffic.md, or None if absent or taken on other sources."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.md")
+    if not os.path.exists(path):
+        return None
+    want = source_hash()
+    for line in open(path):
+        cells = [c.strip() for c in line.strip().strip("|").split("|")]
+        if len(cells) >= 5 and cells[0] == workload and cells[1] == kernel and cells[4] == want:
+            try:
+                return float(cells[3])
+            except ValueError:
+                return None
+    return None
+
+
 def roofline_us(stage, work, peaks):
     """Lower-bound time: slower of tensor time (FP8 at 2x the measured bf16 dense peak for the
     indexer, bf16 for attention) and HBM time at the measured copy bandwidth."""
@@ -180,12 +210,17 @@ class Step:
         self.ws = torch.empty(nws, dtype=torch.uint8, device=device)
         self.out_h = torch.empty(self.out.shape, dtype=torch.bfloat16).pin_memory()
         self.loss_h = torch.empty(1, dtype=torch.float32).pin_memory()
-        self.launches_per_step = 3 + (2 if wl.emit_p else 0) + (1 if self._mla_split() else 0)
+        # the split-KV combine is a separate launch only with more than two splits (two splits
+        # combine inside the attention kernel)
+        self.launches_per_step = 3 + (2 if wl.emit_p else 0) + (1 if self._mla_splits() > 2 else 0)
 
-    def _mla_split(self):
+    def _mla_splits(self):
         wl = self.wl
-        return self.dsa.dsa_workspace_bytes(self.dsa.DSA_OP_SPARSE_MLA_FWD, wl.B, wl.Lq, wl.Lk, wl.k,
-                                            wl.H) > 0 and not wl.emit_p
+        if wl.emit_p:
+            return 1
+        ws = self.dsa.dsa_workspace_bytes(self.dsa.DSA_OP_SPARSE_MLA_FWD, wl.B, wl.Lq, wl.Lk, wl.k, wl.H)
+        per_split = wl.rows * wl.H * (wl.d_v + 1) * 4  # partial O + lse of one split
+        return max(1, ws // per_split) if ws else 1
 
     def run(self, ev=None):
         dsa, d, wl = self.dsa, self.d, self.wl
@@ -331,7 +366,7 @@ def gpu_arm(args, rank, world, device):
         peak_t = peaks["bf16_tflops"] * (2 if dom == "indexer" else 1)
         roof = {"kernel": dom, "bound": "tensor", "achieved": ds["tflops"], "peak": peak_t,
                 "unit": "TFLOP/s", "frac": round(ds["tflops"] / peak_t, 4)}
-    roof["traffic"] = None
+    roof["traffic"] = measured_traffic(wl.name, dom)
     roof["peak_source"] = peaks["source"] + (" (fp8 = 2x measured bf16)" if roof["unit"] == "TFLOP/s" and dom == "indexer" else "")
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
