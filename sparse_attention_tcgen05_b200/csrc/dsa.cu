@@ -8,6 +8,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "../../include/dsa.h"
 #include "indexer.cuh"
@@ -97,6 +98,34 @@ inline dsa_status launch_result() {
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
+// Every kernel of the library is launched as a programmatic dependent of the previous launch in
+// the stream (see pdl_wait in ptx.cuh), optionally as clusters of `cluster` CTAs.
+template <typename... KArgs, typename... Args>
+dsa_status launch(void (*kern)(KArgs...), unsigned grid, unsigned block, size_t smem, cudaStream_t stream,
+                  unsigned cluster, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  unsigned n = 0;
+  attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[n].val.programmaticStreamSerializationAllowed = 1;
+  ++n;
+  if (cluster > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  if (cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...) != cudaSuccess) return DSA_ERR_CUDA;
+  return launch_result();
+}
+
 // ------------------------------------------------------------------------------ indexer
 template <int H_I, int D_I, int G>
 dsa_status launch_indexer(const void* q, const void* kk, const float* w, float* scores, int B,
@@ -138,8 +167,7 @@ dsa_status launch_indexer(const void* q, const void* kk, const float* w, float* 
       cudaSuccess)
     return DSA_ERR_CUDA;
   const int grid = static_cast<int>(std::min<long>(items, sms));
-  kern<<<grid, dsa::indexer::kThreads, Cfg::kSmemBytes, stream>>>(tm_q, tm_k, p);
-  return launch_result();
+  return launch(kern, static_cast<unsigned>(grid), dsa::indexer::kThreads, Cfg::kSmemBytes, stream, 1, tm_q, tm_k, p);
 }
 
 // ------------------------------------------------------------------------------ top-k
@@ -147,20 +175,8 @@ template <int C, int KPT>
 dsa_status launch_topk(const float* scores, int32_t* idx, int B, int Lq, int Lk, int k,
                        cudaStream_t stream) {
   auto kern = dsa::topk::topk_kernel<C, KPT>;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(B) * Lq * C);
-  cfg.blockDim = dim3(dsa::topk::kThreads);
-  cfg.dynamicSmemBytes = 0;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = C;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kern, scores, idx, B, Lq, Lk, k) != cudaSuccess) return DSA_ERR_CUDA;
-  return launch_result();
+  return launch(kern, static_cast<unsigned>(B) * Lq * C, dsa::topk::kThreads, 0, stream, C, scores, idx, B, Lq,
+                Lk, k);
 }
 
 // Keys per CTA for a row split over c CTAs (a multiple of 4, as the kernel computes it).
@@ -256,20 +272,9 @@ dsa_status launch_mla(const void* q, const void* kv, const int32_t* idx, int B, 
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              dsa::mla_pair::kSmemBytes) != cudaSuccess)
       return DSA_ERR_CUDA;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(grid));
-    cfg.blockDim = dim3(dsa::mla_pair::kThreads);
-    cfg.dynamicSmemBytes = dsa::mla_pair::kSmemBytes;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = p.fuse2 ? 4 : 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, kern, tm_main, tm_rope, p) != cudaSuccess) return DSA_ERR_CUDA;
-    if (p.fuse2) return launch_result();
+    const dsa_status st = launch(kern, static_cast<unsigned>(grid), dsa::mla_pair::kThreads, dsa::mla_pair::kSmemBytes,
+                                 stream, p.fuse2 ? 4u : 2u, tm_main, tm_rope, p);
+    if (st != DSA_OK || p.fuse2) return st;
   } else {
     CUtensorMap tm_q;
     if (!encode_2d(&tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, D_QK, static_cast<uint64_t>(rows) * H,
@@ -279,14 +284,15 @@ dsa_status launch_mla(const void* q, const void* kv, const int32_t* idx, int B, 
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) !=
         cudaSuccess)
       return DSA_ERR_CUDA;
-    kern<<<static_cast<unsigned>(grid), dsa::mla::kThreads, Cfg::kSmemBytes, stream>>>(tm_q, p);
+    const dsa_status st = launch(kern, static_cast<unsigned>(grid), dsa::mla::kThreads, Cfg::kSmemBytes, stream, 1,
+                                 tm_q, p);
+    if (st != DSA_OK) return st;
   }
-  if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
   if (sp.n_split > 1) {
     const int cgrid = (rows * H + dsa::mla::kCombineWarps - 1) / dsa::mla::kCombineWarps;
-    dsa::mla::combine_kernel<D_V><<<cgrid, dsa::mla::kCombineWarps * 32, 0, stream>>>(
-        p.part_o, p.part_lse, sp.n_split, rows * H, static_cast<__nv_bfloat16*>(out), lse);
-    return launch_result();
+    return launch(dsa::mla::combine_kernel<D_V>, static_cast<unsigned>(cgrid), dsa::mla::kCombineWarps * 32, 0, stream,
+                  1, static_cast<const float*>(p.part_o), static_cast<const float*>(p.part_lse), sp.n_split, rows * H,
+                  static_cast<__nv_bfloat16*>(out), lse);
   }
   return DSA_OK;
 }
@@ -453,11 +459,11 @@ dsa_status dsa_indexer_kl(const float* scores, const int32_t* idx, const float* 
   const dsa_status ds = current_device(dev);
   if (ds != DSA_OK) return ds;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  dsa::kl::kl_rows_kernel<<<static_cast<unsigned>(rows), dsa::kl::kRowThreads, 0, st>>>(
-      scores, idx, p_sel, Lk, k, per_row);
-  if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
-  dsa::kl::kl_sum_kernel<<<1, dsa::kl::kSumThreads, 0, st>>>(per_row, static_cast<int>(rows), loss);
-  return launch_result();
+  const dsa_status sr = launch(dsa::kl::kl_rows_kernel, static_cast<unsigned>(rows), dsa::kl::kRowThreads, 0, st, 1,
+                               scores, idx, p_sel, Lk, k, per_row);
+  if (sr != DSA_OK) return sr;
+  return launch(dsa::kl::kl_sum_kernel, 1u, dsa::kl::kSumThreads, 0, st, 1, static_cast<const float*>(per_row),
+                static_cast<int>(rows), loss);
 }
 
 dsa_status dsa_indexer_kl_noalloc(const float* scores, const int32_t* idx, const float* p_sel,
@@ -479,11 +485,11 @@ dsa_status dsa_indexer_kl_noalloc(const float* scores, const int32_t* idx, const
   }
   // Every row's term is written before the sum reads it, so the shared array needs no clearing.
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  dsa::kl::kl_rows_kernel<<<static_cast<unsigned>(rows), dsa::kl::kRowThreads, 0, st>>>(
-      scores, idx, p_sel, Lk, k, per_row);
-  if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
-  dsa::kl::kl_sum_kernel<<<1, dsa::kl::kSumThreads, 0, st>>>(per_row, static_cast<int>(rows), loss);
-  return launch_result();
+  const dsa_status sr = launch(dsa::kl::kl_rows_kernel, static_cast<unsigned>(rows), dsa::kl::kRowThreads, 0, st, 1,
+                               scores, idx, p_sel, Lk, k, per_row);
+  if (sr != DSA_OK) return sr;
+  return launch(dsa::kl::kl_sum_kernel, 1u, dsa::kl::kSumThreads, 0, st, 1, static_cast<const float*>(per_row),
+                static_cast<int>(rows), loss);
 }
 
 dsa_status dsa_last_device_status(dsa_stream_t stream) {

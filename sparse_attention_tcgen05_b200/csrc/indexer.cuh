@@ -131,11 +131,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_barrier_init();
     fence_proxy_async_smem();
   }
+  pdl_launch_dependents();
   if (warp == 2) tmem_alloc(tmem_slot, C::kTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();  // first global access below
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer

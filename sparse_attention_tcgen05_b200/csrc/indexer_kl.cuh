@@ -8,6 +8,8 @@
 
 #include <cuda_runtime.h>
 
+#include "ptx.cuh"
+
 namespace dsa {
 namespace kl {
 
@@ -42,6 +44,8 @@ __global__ void __launch_bounds__(kRowThreads)
     kl_rows_kernel(const float* __restrict__ scores, const int32_t* __restrict__ idx,
                    const float* __restrict__ p_sel, int Lk, int k, float* __restrict__ kl_rows) {
   __shared__ float red[32];
+  pdl_launch_dependents();
+  pdl_wait();
   const size_t row = blockIdx.x;
   const float* srow = scores + row * Lk;
   const int32_t* irow = idx + row * k;
@@ -73,6 +77,8 @@ __global__ void __launch_bounds__(kRowThreads)
 __global__ void __launch_bounds__(kSumThreads)
     kl_sum_kernel(const float* __restrict__ kl_rows, int rows, float* __restrict__ loss) {
   __shared__ double red[kSumThreads];
+  pdl_launch_dependents();
+  pdl_wait();
   double acc = 0.0;
   for (int r = threadIdx.x; r < rows; r += kSumThreads) acc += static_cast<double>(kl_rows[r]);
   red[threadIdx.x] = acc;

@@ -36,6 +36,18 @@ __device__ __forceinline__ bool elect_one() {
 }
 
 // ---------------------------------------------------------------------------------------------
+// Programmatic dependent launch.  Every kernel of the library lets the next launch of the stream
+// start as soon as all of its own CTAs are running, and touches global memory only after
+// griddepcontrol.wait, which returns once the previous grid of the stream has completed and
+// its writes are visible (immediately if the kernel was not launched as a dependent).  So the
+// next kernel's launch and its on-chip setup overlap this one's tail, whatever the call order.
+// ---------------------------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// ---------------------------------------------------------------------------------------------
 // mbarrier
 // ---------------------------------------------------------------------------------------------
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {

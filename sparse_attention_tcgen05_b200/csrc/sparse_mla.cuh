@@ -142,11 +142,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_barrier_init();
     fence_proxy_async_smem();
   }
+  pdl_launch_dependents();
   if (warp == 4) tmem_alloc(tmem_slot, C::kTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();  // first global access below
   const uint32_t tmem_o = tmem_base;
   const uint32_t tmem_s = tmem_base + C::kDvCta;
 
@@ -451,6 +453,8 @@ __global__ void __launch_bounds__(kCombineWarps * 32)
                    int rows_h, __nv_bfloat16* __restrict__ out, float* lse) {
   constexpr int kPer = D_V / 32;  // columns per lane
   static_assert(kPer % 2 == 0, "D_V");
+  pdl_launch_dependents();
+  pdl_wait();
   const int rh = blockIdx.x * kCombineWarps + static_cast<int>(threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (rh >= rows_h) return;  // warp-uniform

@@ -181,12 +181,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_barrier_init();
     fence_proxy_async_smem();
   }
+  pdl_launch_dependents();
   if (warp == kMmaWarp) tmem_alloc(tmem_slot, kTmemCols);
   tc_fence_before();
   // the peer's barriers must be initialised before any remote store completes on them
   cluster_barrier();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();  // first global access below
 
   // Effective length: slots after the last valid one in [e0, e1) need no work (same on both).
   {

@@ -101,6 +101,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ uint32_t result[2];
   __shared__ uint32_t totals[2];  // this CTA's (count > T, count == T), read by later ranks
 
+  pdl_launch_dependents();
+  pdl_wait();
   const int row = blockIdx.x / C;
   const uint32_t rank = (C > 1) ? cluster_ctarank() : 0u;
   const int i = row % Lq;
