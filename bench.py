@@ -299,22 +299,30 @@ def gpu_arm(args, rank, world, device):
     for _ in range(args.warmup):
         step.run()
     torch.cuda.synchronize()
-    nev = 5
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(args.steps)]
-    stage_ms = {"indexer": [], "topk": [], "sparse_mla": [], "indexer_kl": []}
+    # Timed region: each step's launches go back to back between one pair of events (events
+    # between the kernels would stop each launch from overlapping the previous kernel's tail).
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
     with ClockSampler(pci_id(device)) as clk:
         for i in range(args.steps):
             flush.fill_(i & 0xFF)  # evict L2 between steps (outside the step's events)
-            step.run(evs[i])
+            evs[i][0].record()
+            step.run()
+            evs[i][1].record()
         torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
-    step_ms = []
-    for e in evs:
-        step_ms.append(e[0].elapsed_time(e[4]))
+    step_ms = [a.elapsed_time(b) for a, b in evs]
+    # Per-stage times (for the stage roofline fractions) from a separate pass of the same steps
+    # with an event between every two launches.
+    stage_ms = {"indexer": [], "topk": [], "sparse_mla": [], "indexer_kl": []}
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+        step.run(e)
+        torch.cuda.synchronize()
         stage_ms["indexer"].append(e[0].elapsed_time(e[1]))
         stage_ms["topk"].append(e[1].elapsed_time(e[2]))
         stage_ms["sparse_mla"].append(e[2].elapsed_time(e[3]))
@@ -379,7 +387,8 @@ def gpu_arm(args, rank, world, device):
         "dtype": "fp8e4m3 indexer, bf16 attention, fp32 accumulate", "data": "synthetic (seeded)",
         "config": {"workload": wl.name, "B": wl.B, "Lq": wl.Lq, "Lk": wl.Lk, "H_I": wl.H_I,
                    "d_I": wl.d_I, "k": wl.k, "H": wl.H, "d_qk": wl.d_qk, "d_v": wl.d_v,
-                   "emit_p_and_kl": wl.emit_p, "l2": "flushed (512 MiB write) between steps, outside the step events"},
+                   "emit_p_and_kl": wl.emit_p, "l2": "flushed (512 MiB write) between steps, outside the step events",
+                   "stage_times": "separate pass with events between launches"},
         "e2e": {"value": wl.rows * world / (e2e_ms / 1e3), "unit": "query-tokens/s",
                 "h2d_bytes_per_step": step.h2d_bytes(), "d2h_bytes_per_step": step.d2h_bytes()},
         "gpu_launches": step.launches_per_step * args.steps,

@@ -13,17 +13,18 @@
 // mbarrier); both then hold the same full S (fp32 addition commutes), take the same softmax
 // decisions and accumulate O for their own 256 value dims.
 //
-// Tensor memory (512 columns): O [0, 256) fp32, S 2 x 32 fp32 [256, 320), and this CTA's
-// slice of Q, 128 heads x 288 bf16, as the A operand of S = Q K^T [320, 464).  Keeping Q in
+// Tensor memory (512 columns): O [0, 256) fp32, S 2 x 32 fp32 [256, 320), this CTA's slice of
+// Q, 128 heads x 288 bf16, as the A operand of S = Q K^T [320, 464), and P 2 x 16 [464, 496)
+// (bf16, the A operand of O += P V).  Keeping Q in
 // tensor memory means a 32-wide S block only streams its 18 KB gathered tile from shared
 // memory, and frees shared memory for an 8-deep gather ring.
 //
 // Pipeline (per CTA, blocks of 32 selected entries; a p sweep revisits every block):
 //   gather warps   TMA tile::gather4: 4 selected rows per instruction, landing in the
-//                  swizzled K-major tiles the MMA reads (6 stages, 40 instructions a block).
-//                  A single issuing warp caps the gather near 9 GB/s per SM, so six warps
-//                  take turns by block (warp w always refills stage w).
-//   MMA thread     polls: S(j) = Q K_j^T as soon as block j and an S buffer are free;
+//                  swizzled K-major tiles the MMA reads (3 stages of a pair of blocks, 80
+//                  instructions each); all seven warps share every stage.
+//   MMA thread     polls: S = Q K^T of a pair of blocks (N = 64) as soon as its stage landed
+//                  and the previous pair's S was read;
 //                  O += P(i) V_i as soon as P(i) is written (never waits behind a late gather)
 //   softmax        two warpgroups on the same 128 TMEM lanes (thread = head row) take turns by
 //                  block, so two blocks are in flight: each loads its partial S, ships it to the
@@ -44,35 +45,35 @@ using mla::Params;
 using mla::pack_bf16x2;
 using mla::named_bar_sync;
 
-constexpr int kBN = 32;             // selected entries per block
-constexpr int kStages = 6;          // gather ring depth (a multiple of kGatherWarps)
+constexpr int kBN = 32;             // selected entries per softmax block
+constexpr int kPairN = 2 * kBN;     // entries per gathered stage and per S = Q K^T (MMA N = 64)
+constexpr int kStages = 3;          // gather ring depth (pairs of blocks)
 constexpr int kRecvSlots = 4;       // partial-S receive slots (see the exchange argument below)
-constexpr int kThreads = 480;       // warps 0-7 softmax, 8 MMA, 9-14 gather
+constexpr int kThreads = 512;       // warps 0-7 softmax, 8 MMA, 9-15 gather
 constexpr int kSoftmaxThreads = 256;  // two warpgroups taking turns by block
 constexpr int kMmaWarp = 8;
 constexpr int kGatherWarp0 = 9;
-constexpr int kGatherWarps = 6;
+constexpr int kGatherWarps = 7;
 constexpr int kDQK = 576, kDV = 512, kDvCta = 256, kRopeCta = 32;
 constexpr int kDimsCta = kDvCta + kRopeCta;         // 288 key dims per CTA
-constexpr int kMainBox = kBN * 128;                 // 32 entries x 64 dims (SW128)
-constexpr int kRopeTile = kBN * 64;                 // 32 entries x 32 dims (SW64)
-constexpr int kKvStage = 4 * kMainBox + kRopeTile;  // 18 KB
-constexpr int kPBytes = 128 * kBN * 2;
+constexpr int kMainBox = kPairN * 128;              // 64 entries x 64 dims (SW128)
+constexpr int kRopeTile = kPairN * 64;              // 64 entries x 32 dims (SW64)
+constexpr int kKvStage = 4 * kMainBox + kRopeTile;  // 36 KB
 constexpr int kXSlot = 128 * kBN * 4;               // one partial S (fp32, 16 KB)
 constexpr int kOffKV = 0;
 constexpr int kOffX = kOffKV + kStages * kKvStage;  // [kRecvSlots] the peer's partials
 constexpr int kOffXs = kOffX + kRecvSlots * kXSlot; // [2] own partials staged for the bulk copy
-constexpr int kOffP = kOffXs + 2 * kXSlot;
-constexpr int kOffRed = kOffP + 2 * kPBytes;      // [2 groups][4 warps][32] p partial sums
-constexpr int kOffRef = kOffRed + 2 * 4 * 32 * 4;  // [2][128] per-row reference of a block
+constexpr int kOffRef = kOffXs + 2 * kXSlot;      // [2][128] per-row reference of a block
+constexpr int kOffRed = kOffRef;                   // [2 groups][4 warps][32] p partial sums: the p
+                                                   // sweep starts after every reference was read
 constexpr int kOffFin = kOffRef + 2 * 128 * 4;     // [2 groups][2][128] final (l, reference)
 constexpr int kOffBar = kOffFin + 2 * 2 * 128 * 4;
 constexpr int kNumBars = 2 * kStages + 8 + kRecvSlots + 3;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kSmemBytes = kOffMisc + 64 + 1024;
 constexpr int kTmemCols = 512;
-constexpr uint32_t kTmemO = 0, kTmemS = 256, kTmemQ = 320;
-constexpr uint32_t kIdescQK = make_idesc(1, 1, false, false, 128, kBN);
+constexpr uint32_t kTmemO = 0, kTmemS = 256, kTmemQ = 320, kTmemP = 464;
+constexpr uint32_t kIdescQK = make_idesc(1, 1, false, false, 128, kPairN);
 constexpr uint32_t kIdescPV = make_idesc(1, 1, false, true, 128, kDvCta);
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleLog2 = 8.0f;
@@ -82,13 +83,13 @@ constexpr int kBarRed0 = 3;  // p sweep partial sums
 constexpr int kBarFin = 5;   // final normaliser of both groups
 static_assert(kSmemBytes <= 232448, "shared memory");
 static_assert(kKvStage % 1024 == 0, "stage alignment (128B-swizzle atoms)");
-// A gather warp waits on a stage's barrier for the phase of its own previous block there; if
-// the stage also served another warp's blocks, that warp could see the phase two steps ahead.
-static_assert(kStages % kGatherWarps == 0, "a stage must always cycle through the same gather warp");
-static_assert(kTmemQ + kDimsCta / 2 <= kTmemCols, "tensor memory");
+static_assert(kGatherWarps * 12 >= 80, "every gather operation of a stage has a lane");
+static_assert(kTmemQ + kDimsCta / 2 <= kTmemP && kTmemP + 2 * kBN / 2 <= kTmemCols, "tensor memory");
 
-// S = Q K^T over this CTA's 288 key dims: 16 K-steps over the four 64-dim boxes (SW128) and 2
-// over the 32 rope dims (SW64).  A (Q) comes from tensor memory, 8 columns per K-step.
+// S = Q K^T of a pair of blocks (64 entries, N = 64: an M = 128, K = 16 MMA costs the same ~51
+// cycles at N = 32 and N = 64, and reaches full rate only from N = 128) over this CTA's 288 key
+// dims: 16 K-steps over the four 64-dim boxes (SW128) and 2 over the 32 rope dims (SW64).  A (Q)
+// comes from tensor memory, 8 columns per K-step; D is the pair's 64 S columns.
 __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_tmem, uint32_t kv_addr) {
   const uint64_t kb = make_smem_desc(kv_addr, 16, 1024, kSw128);
   const uint64_t rb = make_smem_desc(kv_addr + 4 * kMainBox, 16, 512, kSw64);
@@ -103,16 +104,15 @@ __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_tmem, uint3
     mma_f16_ts(d_tmem, q_tmem + 8 * (16 + kk), rb + static_cast<uint64_t>((kk * 32) >> 4), kIdescQK, 1u);
 }
 
-// O (+)= P V: A = P (128 x 32 bf16, SW64 K-major), B = the gathered value dims read MN-major
-// (4 boxes of 64 dims at LBO = one box), 2 K-steps of 16 entries.
-__device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_addr, uint32_t kv_addr,
-                                         bool first) {
-  const uint64_t pd = make_smem_desc(p_addr, 16, 512, kSw64);
-  const uint64_t vd = make_smem_desc(kv_addr, kMainBox, 1024, kSw128);
+// O (+)= P V of one block: A = P (128 x 32 bf16 in tensor memory, 16 columns, written by the
+// softmax threads), B = the block's half (rows 32 half.. of each box) of the gathered value dims
+// read MN-major (4 boxes of 64 dims at LBO = one box), 2 K-steps of 16 entries.
+__device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_t kv_addr, int half, bool first) {
+  const uint64_t vd = make_smem_desc(kv_addr + half * (kBN * 128), kMainBox, 1024, kSw128);
 #pragma unroll
   for (int kk = 0; kk < kBN / 16; ++kk)
-    mma_f16_ss(o_tmem, pd + static_cast<uint64_t>((kk * 32) >> 4),
-               vd + static_cast<uint64_t>((kk * 16 * 128) >> 4), kIdescPV, (!first || kk > 0) ? 1u : 0u);
+    mma_f16_ts(o_tmem, p_tmem + 8 * kk, vd + static_cast<uint64_t>((kk * 16 * 128) >> 4), kIdescPV,
+               (!first || kk > 0) ? 1u : 0u);
 }
 
 // The 32 idx slots of block `blk` as seen by lane `lane` (-1 past the effective length).
@@ -128,7 +128,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sKV = smem + kOffKV;
-  uint8_t* sP = smem + kOffP;
   float* sX = reinterpret_cast<float*>(smem + kOffX);
   uint8_t* sXs = smem + kOffXs;
   float* sRed = reinterpret_cast<float*>(smem + kOffRed);
@@ -137,8 +136,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
   uint64_t* kv_full = bars;                 // [kStages] expect_tx + the gathered bytes
   uint64_t* kv_empty = bars + kStages;      // [kStages] MMA commit
-  uint64_t* s_full = bars + 2 * kStages;    // [2] MMA commit
-  uint64_t* s_empty = s_full + 2;           // [2] 128 arrivals of the block's warpgroup
+  uint64_t* s_full = bars + 2 * kStages;    // [1 used] MMA commit of a pair's S
+  uint64_t* s_empty = s_full + 2;           // [2] per half of a pair: 128 arrivals of its warpgroup
   uint64_t* p_full = s_full + 4;            // [2] 128 arrivals of the block's warpgroup
   uint64_t* o_done = s_full + 6;            // [2] MMA commit (PV of blocks i, i % 2)
   uint64_t* x_full = s_full + 8;            // [kRecvSlots] own expect_tx + the peer's bytes
@@ -210,26 +209,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!mbar_wait(q_ready, 0, abort_flag, 60)) goto done;
       tc_fence_after();
       const uint32_t q_tmem = tmem_base + kTmemQ;
-      int nq = 0, np = 0;  // next S block to compute, next PV block
+      const int npairs = (total + 1) / 2;
+      int nq = 0, np = 0;  // next pair to compute S for, next block to run PV for
       uint64_t t_idle = 0;
-      while (nq < total || np < nblk) {
+      while (nq < npairs || np < nblk) {
         bool progress = false;
-        if (nq < total && mbar_test_wait(&kv_full[nq % kStages], (nq / kStages) & 1) &&
-            mbar_test_wait(&s_empty[nq & 1], ((nq >> 1) & 1) ^ 1)) {
+        // S of pair nq once its stage has landed and both halves of pair nq-1 were read
+        if (nq < npairs && mbar_test_wait(&kv_full[nq % kStages], (nq / kStages) & 1) &&
+            mbar_test_wait(&s_empty[0], (nq & 1) ^ 1) && mbar_test_wait(&s_empty[1], (nq & 1) ^ 1)) {
           tc_fence_after();
           const int st = nq % kStages;
-          issue_qk(tmem_base + kTmemS + (nq & 1) * kBN, q_tmem, smem_u32(sKV + st * kKvStage));
-          mma_commit(&s_full[nq & 1]);
-          if (nq >= nblk) mma_commit(&kv_empty[st]);  // p sweep: no PV reads this block
+          issue_qk(tmem_base + kTmemS, q_tmem, smem_u32(sKV + st * kKvStage));
+          mma_commit(&s_full[0]);
+          if (2 * nq >= nblk) mma_commit(&kv_empty[st]);  // no PV reads this stage (p sweep)
           ++nq;
           progress = true;
         }
-        if (np < nblk && np < nq && mbar_test_wait(&p_full[np & 1], (np >> 1) & 1)) {
+        // PV of block np; the stage is released after the last MMA that reads it
+        if (np < nblk && (np >> 1) < nq && mbar_test_wait(&p_full[np & 1], (np >> 1) & 1)) {
           tc_fence_after();
-          const int st = np % kStages;
-          issue_pv(tmem_base + kTmemO, smem_u32(sP + (np & 1) * kPBytes), smem_u32(sKV + st * kKvStage),
-                   np == 0);
-          mma_commit(&kv_empty[st]);
+          const int st = (np >> 1) % kStages;
+          issue_pv(tmem_base + kTmemO, tmem_base + kTmemP + (np & 1) * (kBN / 2), smem_u32(sKV + st * kKvStage),
+                   np & 1, np == 0);
+          if ((np & 1) || np + 1 >= nblk) mma_commit(&kv_empty[st]);
           mma_commit(&o_done[np & 1]);
           ++np;
           progress = true;
@@ -252,53 +254,60 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= kGatherWarp0) {
     // ------------------------------------------------------------------ gather (TMA)
-    // Gather warp w takes blocks j = w, w + 6, ... (all of them in stage w)  Lane r holds the block's r-th index; lane
-    // g < 8 gathers entries 4g..4g+3: the four 64-dim boxes of this CTA's value dims and its
-    // 32 rope dims.  Invalid slots point one row past
-    // the tensor, which the TMA fills with zeros.
+    // A stage holds a pair of blocks (64 entries): 80 gather4 operations (16 groups of four
+    // entries x the four 64-dim boxes of this CTA's value dims and its 32 rope dims).  All gather
+    // warps share every stage - warp w issues operations w, w + 7, ... (lanes 0-11) - since one
+    // warp issues them about 80 cycles apart.  Every warp waits on the same stage barrier for
+    // every pair; none can run two phases ahead, since pair jp + kStages needs pair jp consumed,
+    // which needs pair jp landed.  Lane r holds the r-th index of each block of the pair;
+    // invalid slots (and the missing half of an odd last pair) point one row past the tensor,
+    // which the TMA fills with zeros.
     const int row0 = b * p.Lk;
     const int oob = p.B * p.Lk;
-    const int g = lane & 7;
-    const int main0 = static_cast<int>(rank) * kDvCta;         // first value dim of this CTA
-    const int rope0 = kDV + static_cast<int>(rank) * kRopeCta;  // first rope dim of this CTA
     const int w = warp - kGatherWarp0;
-    int next_s = (w < total) ? block_slot(idx_row, e0, len, w < nblk ? w : w - nblk, lane) : -1;
-    int issued = w;  // one past the last block this warp issued
+    const int op = w + kGatherWarps * lane;  // this lane's operation of each stage
+    const bool has_op = lane < 12 && op < 80;
+    const int g = has_op ? op / 5 : 0;       // entry group: entries 4g..4g+3 of the pair
+    const int bx = has_op ? op % 5 : 0;      // 0-3: value box, 4: rope dims
+    const int x0 = bx < 4 ? static_cast<int>(rank) * kDvCta + bx * 64 : kDV + static_cast<int>(rank) * kRopeCta;
+    const CUtensorMap* tmap = bx < 4 ? &tm_main : &tm_rope;
+    const uint32_t dst_off = bx < 4 ? static_cast<uint32_t>(bx * kMainBox + g * 512) : static_cast<uint32_t>(4 * kMainBox + g * 256);
+    const int npairs = (total + 1) / 2;
+    auto slot_of = [&](int j) { return j < total ? block_slot(idx_row, e0, len, j < nblk ? j : j - nblk, lane) : -1; };
+    int next_lo = (total > 0) ? slot_of(0) : -1, next_hi = (total > 1) ? slot_of(1) : -1;
+    int issued = 0;
     if (lane == 0) {
       tma_prefetch_desc(&tm_main);
       tma_prefetch_desc(&tm_rope);
     }
-    for (int j = w; j < total; j += kGatherWarps) {
-      const int st = j % kStages;
-      const bool got = mbar_wait(&kv_empty[st], ((j / kStages) & 1) ^ 1, abort_flag, 62);
+    for (int jp = 0; jp < npairs; ++jp) {
+      const int st = jp % kStages;
+      const bool got = mbar_wait(&kv_empty[st], ((jp / kStages) & 1) ^ 1, abort_flag, 62);
       if (!__all_sync(0xFFFFFFFFu, got)) break;  // the shuffles below need the whole warp
-      const int my_s = next_s;
-      const int jn = j + kGatherWarps;
-      if (jn < total) next_s = block_slot(idx_row, e0, len, jn < nblk ? jn : jn - nblk, lane);
-      if (my_s >= p.Lk) record_bad_index();
-      const int y = (static_cast<unsigned>(my_s) < static_cast<unsigned>(p.Lk)) ? row0 + my_s : oob;
-      const int y0 = __shfl_sync(0xFFFFFFFFu, y, 4 * g);
-      const int y1 = __shfl_sync(0xFFFFFFFFu, y, 4 * g + 1);
-      const int y2 = __shfl_sync(0xFFFFFFFFu, y, 4 * g + 2);
-      const int y3 = __shfl_sync(0xFFFFFFFFu, y, 4 * g + 3);
-      if (lane == 0) mbar_arrive_expect_tx(&kv_full[st], kKvStage);
-      __syncwarp();
-      if (lane < 8) {
-        uint8_t* dst = sKV + st * kKvStage;
-#pragma unroll
-        for (int bx = 0; bx < 4; ++bx)
-          tma_gather4(dst + bx * kMainBox + g * 512, &tm_main, &kv_full[st], main0 + bx * 64, y0, y1, y2, y3);
-        tma_gather4(dst + 4 * kMainBox + g * 256, &tm_rope, &kv_full[st], rope0, y0, y1, y2, y3);
+      const int s_lo = next_lo, s_hi = next_hi;
+      if (jp + 1 < npairs) {
+        next_lo = slot_of(2 * jp + 2);
+        next_hi = slot_of(2 * jp + 3);
       }
-      issued = j + 1;
+      if (s_lo >= p.Lk || s_hi >= p.Lk) record_bad_index();
+      const int y_lo = (static_cast<unsigned>(s_lo) < static_cast<unsigned>(p.Lk)) ? row0 + s_lo : oob;
+      const int y_hi = (static_cast<unsigned>(s_hi) < static_cast<unsigned>(p.Lk)) ? row0 + s_hi : oob;
+      const int src = 4 * (g & 7);
+      int yv[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int a = __shfl_sync(0xFFFFFFFFu, y_lo, src + i);
+        const int c = __shfl_sync(0xFFFFFFFFu, y_hi, src + i);
+        yv[i] = g < 8 ? a : c;
+      }
+      if (w == 0 && lane == 0) mbar_arrive_expect_tx(&kv_full[st], kKvStage);
+      if (has_op) tma_gather4(sKV + st * kKvStage + dst_off, tmap, &kv_full[st], x0, yv[0], yv[1], yv[2], yv[3]);
+      issued = jp + 1;
     }
     // Nothing of ours may still be landing when the CTA exits.  On the normal path the MMA
-    // consumed every block; after an abort, wait (bounded) for this warp's last blocks.
-    if (lane == 0 && *abort_flag) {
-      const int lo = max(w, issued - kStages);
-      for (int j = lo + (w - lo % kGatherWarps + kGatherWarps) % kGatherWarps; j < issued; j += kGatherWarps)
-        mbar_drain(&kv_full[j % kStages], (j / kStages) & 1);
-    }
+    // consumed every stage; after an abort, wait (bounded) for the last stages.
+    if (w == 0 && lane == 0 && *abort_flag)
+      for (int j = max(0, issued - kStages); j < issued; ++j) mbar_drain(&kv_full[j % kStages], (j / kStages) & 1);
   } else {
     // ------------------------------------------------------------------ softmax / epilogue
     // Warpgroup wg handles blocks q = wg, wg + 2, ... (thread = head row over all 32 columns),
@@ -372,7 +381,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (wtid == 0) bulk_wait_read_all();
       named_bar_sync(bar_xs, 128);
       uint32_t v[32];
-      if (ok && !mbar_wait(&s_full[q & 1], (q >> 1) & 1, abort_flag, 63)) ok = false;
+      if (ok && !mbar_wait(&s_full[0], (q >> 1) & 1, abort_flag, 63)) ok = false;
       ok = __all_sync(0xFFFFFFFFu, ok);  // tcgen05.ld is warp-collective
       if (ok) {
         tc_fence_after();
@@ -559,12 +568,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const float2 r2 = add2(add2(rs[0], rs[1]), add2(rs[2], rs[3]));
           l += r2.x + r2.y;
-          uint8_t* pbuf = sP + pb * kPBytes;  // row h: 64 B, 64B-swizzled
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-            *reinterpret_cast<uint4*>(pbuf + swizzled_offset(h, j, 64)) =
-                make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
-          fence_proxy_async_smem();
+          tmem_st_32x32b_x16(tm + kTmemP + pb * (kBN / 2), pk);  // row h, 32 bf16 = 16 columns
+          tmem_st_wait();
           tc_fence_before();
           mbar_arrive(&p_full[pb]);
         }
