@@ -268,12 +268,19 @@ dsa_status launch_mla(const void* q, const void* kv, const int32_t* idx, int B, 
         !encode_2d(&tm_rope, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kv, D_QK, static_cast<uint64_t>(B) * Lk,
                    static_cast<uint64_t>(D_QK) * 2, 32, 1, CU_TENSOR_MAP_SWIZZLE_64B))
       return DSA_ERR_CUDA;
+    // q as [rows * H, 576]: 128 head rows x 64 dims (SW128) and x the 32 rope dims (SW64)
+    CUtensorMap tm_q_main, tm_q_rope;
+    if (!encode_2d(&tm_q_main, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, D_QK, static_cast<uint64_t>(rows) * H,
+                   static_cast<uint64_t>(D_QK) * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_2d(&tm_q_rope, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, D_QK, static_cast<uint64_t>(rows) * H,
+                   static_cast<uint64_t>(D_QK) * 2, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B))
+      return DSA_ERR_CUDA;
     auto kern = dsa::mla_pair::sparse_mla_pair_kernel;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              dsa::mla_pair::kSmemBytes) != cudaSuccess)
       return DSA_ERR_CUDA;
     const dsa_status st = launch(kern, static_cast<unsigned>(grid), dsa::mla_pair::kThreads, dsa::mla_pair::kSmemBytes,
-                                 stream, p.fuse2 ? 4u : 2u, tm_main, tm_rope, p);
+                                 stream, p.fuse2 ? 4u : 2u, tm_main, tm_rope, tm_q_main, tm_q_rope, p);
     if (st != DSA_OK || p.fuse2) return st;
   } else {
     CUtensorMap tm_q;

@@ -68,7 +68,7 @@ constexpr int kOffRed = kOffRef;                   // [2 groups][4 warps][32] p 
                                                    // sweep starts after every reference was read
 constexpr int kOffFin = kOffRef + 2 * 128 * 4;     // [2 groups][2][128] final (l, reference)
 constexpr int kOffBar = kOffFin + 2 * 2 * 128 * 4;
-constexpr int kNumBars = 2 * kStages + 8 + kRecvSlots + 3;
+constexpr int kNumBars = 2 * kStages + 8 + kRecvSlots + 4;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kSmemBytes = kOffMisc + 64 + 1024;
 constexpr int kTmemCols = 512;
@@ -83,6 +83,11 @@ constexpr int kBarRed0 = 3;  // p sweep partial sums
 constexpr int kBarFin = 5;   // final normaliser of both groups
 static_assert(kSmemBytes <= 232448, "shared memory");
 static_assert(kKvStage % 1024 == 0, "stage alignment (128B-swizzle atoms)");
+// This CTA's Q slice (128 head rows x 288 dims) is staged by TMA in gather stages 1.. before the
+// first gathers need them: four 64-dim boxes (SW128) and the 32 rope dims (SW64).
+constexpr int kQBox = 128 * 128;
+constexpr int kQBytes = 4 * kQBox + 128 * 64;
+static_assert(kQBytes <= (kStages - 1) * kKvStage, "Q staging fits in stages 1..");
 static_assert(kGatherWarps * 12 >= 80, "every gather operation of a stage has a lane");
 static_assert(kTmemQ + kDimsCta / 2 <= kTmemP && kTmemP + 2 * kBN / 2 <= kTmemCols, "tensor memory");
 
@@ -123,7 +128,9 @@ __device__ __forceinline__ int block_slot(const int32_t* idx_row, int e0, int le
 
 __global__ void __launch_bounds__(kThreads, 1)
     sparse_mla_pair_kernel(const __grid_constant__ CUtensorMap tm_main,
-                           const __grid_constant__ CUtensorMap tm_rope, const Params p) {
+                           const __grid_constant__ CUtensorMap tm_rope,
+                           const __grid_constant__ CUtensorMap tm_q_main,
+                           const __grid_constant__ CUtensorMap tm_q_rope, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -143,6 +150,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* x_full = s_full + 8;            // [kRecvSlots] own expect_tx + the peer's bytes
   uint64_t* q_ready = x_full + kRecvSlots;  // 256 softmax arrivals: Q is in tensor memory
   uint64_t* ref_full = q_ready + 1;         // [2] 128 arrivals: a block's reference is published
+  uint64_t* q_full = ref_full + 2;          // expect_tx + the staged Q slice
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
   int* s_len = reinterpret_cast<int*>(smem + kOffMisc + 8);
@@ -175,6 +183,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < kRecvSlots; ++i) mbar_init(&x_full[i], 1);
     mbar_init(q_ready, kSoftmaxThreads);
+    mbar_init(q_full, 1);
     *abort_flag = 0;
     *s_len = 0;
     fence_barrier_init();
@@ -188,6 +197,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   pdl_wait();  // first global access below
+  if (threadIdx.x == kMmaWarp * 32) {
+    // Q rows row*H .. row*H+127 (rows past H belong to other queries or lie outside the tensor
+    // and are zeroed by the readers), this CTA's dims
+    uint8_t* qs = sKV + kKvStage;
+    const int y = row * p.H;
+    mbar_arrive_expect_tx(q_full, kQBytes);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) tma_load_2d(qs + i * kQBox, &tm_q_main, q_full, static_cast<int>(rank) * kDvCta + i * 64, y);
+    tma_load_2d(qs + 4 * kQBox, &tm_q_rope, q_full, kDV + static_cast<int>(rank) * kRopeCta, y);
+  }
 
   // Effective length: slots after the last valid one in [e0, e1) need no work (same on both).
   {
@@ -282,7 +301,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int jp = 0; jp < npairs; ++jp) {
       const int st = jp % kStages;
-      const bool got = mbar_wait(&kv_empty[st], ((jp / kStages) & 1) ^ 1, abort_flag, 62);
+      // stages 1.. hold the staged Q until it is in tensor memory
+      bool got = jp != 1 || mbar_wait(q_ready, 0, abort_flag, 66);
+      got = got && mbar_wait(&kv_empty[st], ((jp / kStages) & 1) ^ 1, abort_flag, 62);
       if (!__all_sync(0xFFFFFFFFu, got)) break;  // the shuffles below need the whole warp
       const int s_lo = next_lo, s_hi = next_hi;
       if (jp + 1 < npairs) {
@@ -335,30 +356,32 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* stg_row = sXs + wg * kXSlot + h * (kBN * 4);  // this group's staging slot, row h
     bool ok = true;
 
-    if (total > 0) {
-      // This CTA's 288 dims of Q into tensor memory: dims [8j, 8j+8) of the slice -> columns
-      // [4j, 4j+4), in 9 groups of 16 columns (warpgroup 0 takes groups 0-4, 1 takes 5-8).
-      // Heads >= H get zeros.
-      // All of a thread's loads are issued before the first store, so the prologue costs one
-      // memory round trip rather than five.
-      const __nv_bfloat16* qrow = p.q + orow * kDQK;
+    // This CTA's 288 dims of Q into tensor memory: dims [8j, 8j+8) of the slice -> columns
+    // [4j, 4j+4), in 9 groups of 16 columns (warpgroup 0 takes groups 0-4, 1 takes 5-8), read
+    // from the TMA-staged slice (row h of a box; 16-byte chunk c sits at c ^ (h & 7) in a
+    // 128-byte row, at c ^ ((h >> 1) & 3) in a 64-byte rope row).  Heads >= H get zeros.  The
+    // staged slice is waited for even with no work, so no copy is in flight at exit.
+    if (!mbar_wait(q_full, 0, abort_flag, 65)) {
+      ok = false;
+      if (threadIdx.x == 0) mbar_drain(q_full, 0);  // let the staged copy land before exit
+    }
+    if (ok && total > 0) {
+      const uint8_t* qs = sKV + kKvStage;
       const int g0 = wg * 5, ng = wg == 0 ? 5 : 4;
-      uint4 v[20];
-#pragma unroll
-      for (int i = 0; i < 20; ++i) {
-        const int j = g0 * 4 + i;
-        const int d = j < 32 ? static_cast<int>(rank) * kDvCta + j * 8
-                             : kDV + static_cast<int>(rank) * kRopeCta + (j - 32) * 8;
-        v[i] = (head_ok && i < ng * 4) ? __ldg(reinterpret_cast<const uint4*>(qrow + d)) : make_uint4(0u, 0u, 0u, 0u);
-      }
 #pragma unroll
       for (int gi = 0; gi < 5; ++gi) {
         if (gi < ng) {
-          const uint32_t r[16] = {v[4 * gi].x,     v[4 * gi].y,     v[4 * gi].z,     v[4 * gi].w,
-                                  v[4 * gi + 1].x, v[4 * gi + 1].y, v[4 * gi + 1].z, v[4 * gi + 1].w,
-                                  v[4 * gi + 2].x, v[4 * gi + 2].y, v[4 * gi + 2].z, v[4 * gi + 2].w,
-                                  v[4 * gi + 3].x, v[4 * gi + 3].y, v[4 * gi + 3].z, v[4 * gi + 3].w};
-          tmem_st_32x32b_x16(tm + kTmemQ + (g0 + gi) * 16, r);
+          const int gg = g0 + gi;
+          uint4 v[4];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const uint8_t* src = gg < 8 ? qs + (gg >> 1) * kQBox + h * 128 + ((((gg & 1) * 4 + c) ^ (h & 7)) << 4)
+                                        : qs + 4 * kQBox + h * 64 + ((c ^ ((h >> 1) & 3)) << 4);
+            v[c] = head_ok ? *reinterpret_cast<const uint4*>(src) : make_uint4(0u, 0u, 0u, 0u);
+          }
+          const uint32_t r[16] = {v[0].x, v[0].y, v[0].z, v[0].w, v[1].x, v[1].y, v[1].z, v[1].w,
+                                  v[2].x, v[2].y, v[2].z, v[2].w, v[3].x, v[3].y, v[3].z, v[3].w};
+          tmem_st_32x32b_x16(tm + kTmemQ + gg * 16, r);
         }
       }
       tmem_st_wait();
