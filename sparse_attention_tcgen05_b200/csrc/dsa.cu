@@ -175,7 +175,10 @@ template <int C, int KPT>
 dsa_status launch_topk(const float* scores, int32_t* idx, int B, int Lq, int Lk, int k,
                        cudaStream_t stream) {
   auto kern = dsa::topk::topk_kernel<C, KPT>;
-  return launch(kern, static_cast<unsigned>(B) * Lq * C, dsa::topk::kThreads, 0, stream, C, scores, idx, B, Lq,
+  constexpr int smem = dsa::topk::dyn_smem_bytes<KPT>();
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  return launch(kern, static_cast<unsigned>(B) * Lq * C, dsa::topk::kThreads, smem, stream, C, scores, idx, B, Lq,
                 Lk, k);
 }
 

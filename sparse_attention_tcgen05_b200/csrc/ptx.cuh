@@ -169,6 +169,16 @@ __device__ __forceinline__ void bulk_copy_to_peer(uint32_t remote_dst, uint32_t 
       : "memory");
 }
 
+// Asynchronous bulk copy of `bytes` (multiple of 16, both addresses 16-byte aligned) from global
+// memory into this CTA's shared memory; completion is counted as transaction bytes on `bar`.
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(gsrc)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
 // Asynchronous 16-byte store into another CTA's shared memory of the cluster; its bytes count
 // as completed transactions on that CTA's mbarrier (no fence needed on the sending side).
 __device__ __forceinline__ void st_async_v4(uint32_t remote_addr, float a, float b, float c, float d,

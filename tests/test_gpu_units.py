@@ -86,6 +86,7 @@ def _topk_case(dsa, scores_np, Lq, k):
     (64, 1, 16384, 2048, 7),     # 4-CTA clusters
     (8, 1, 40000, 1000, 1000),   # 8-CTA clusters, slice > one block of threads
     (1, 4, 70000, 4096, 9),      # longest k, 4-CTA by length
+    (3, 2, 9999, 512, 20),       # rows not 16-byte aligned: scalar copy into the load stage
 ])
 def test_topk_exact_with_ties(dsa, B, Lq, Lk, k, levels):
     rng = np.random.default_rng(B * 7 + Lk)
