@@ -11,8 +11,8 @@
 //      with their positions into every CTA of the cluster, together with each CTA's count of
 //      keys above d1; after one cluster barrier every CTA settles the two lower digits on the
 //      candidates alone, with no further cluster traffic;
-//   3. if the candidates overflow the buffer (heavy ties), the two lower digits are settled over
-//      the whole slices instead, one cluster round per digit.
+//   3. if the candidates overflow the buffer (heavy ties), or the row has a single CTA, the two
+//      lower digits are settled over the whole slices instead, one cluster round per digit.
 // T and the number r of T-ties to keep fix the set exactly.  The selected positions are marked
 // in bitmaps; exclusive scans of the per-word counts of (key > T, key == T) give every selected
 // position its place in ascending order.
@@ -313,64 +313,68 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr uint32_t kCap = kCandBytes / sizeof(uint2);
   const uint32_t lo1 = d1 << 21, hi1 = lo1 | 0x1FFFFFu;  // the keys of digit d1 (real keys: d1 >= 3)
   uint32_t mabove = 0u, mcand = 0u;                      // bit 4c + e: key e of chunk c
+  uint32_t nc = 0u;     // this thread's candidates
+  uint32_t cbase = 0u;  // slot of this thread's first candidate in the own buffer
+  if constexpr (C > 1) {  // a single CTA settles digits 2 and 3 over its slice (no cluster round to save)
 #pragma unroll
-  for (int c = 0; c < kCpr; ++c) {
-    const uint4 q = stk[tid + kThreads * c];
-    const uint32_t kq[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      mabove |= (kq[e] > hi1 ? 1u : 0u) << (4 * c + e);
-      mcand |= (kq[e] >= lo1 && kq[e] <= hi1 ? 1u : 0u) << (4 * c + e);
-    }
-  }
-  const uint32_t above = __popc(mabove), nc = __popc(mcand);
-  uint32_t cbase;  // slot of this thread's first candidate in the own buffer
-  {
-    // This CTA's list: reserve room in every CTA's buffer, write it into the own buffer, then
-    // copy it to the peers.
-    const uint2 ex = block_exclusive2(nc, above, red);
-    if (tid == kThreads - 1) {
-      const uint32_t tot_c = ex.x + nc, tot_a = ex.y + above;
-      uint32_t o[C];  // every reservation in flight before the first result is used
-#pragma unroll
-      for (int r = 0; r < C; ++r) o[r] = (C > 1) ? atom_add_peer(&n_cand, r, tot_c) : atomicAdd(&n_cand, tot_c);
-#pragma unroll
-      for (int r = 0; r < C; ++r) {
-        if (C > 1)
-          st_peer_u32(&above_of[rank], r, tot_a);
-        else
-          above_of[0] = tot_a;
-      }
-#pragma unroll
-      for (int r = 0; r < C; ++r) offs[r] = o[r];
-      offs[kMaxCluster] = tot_c;
-    }
-    __syncthreads();
-    cbase = offs[rank] + ex.x;
-    uint32_t s = cbase;
-    for (uint32_t cm = mcand; cm != 0u;) {  // only the chunks holding candidates
-      const int c = (__ffs(cm) - 1) >> 2;
-      const uint32_t nib = (cm >> (4 * c)) & 0xFu;
-      cm &= ~(0xFu << (4 * c));
-      const int g = tid + kThreads * c;
-      const uint4 q = stk[g];
+    for (int c = 0; c < kCpr; ++c) {
+      const uint4 q = stk[tid + kThreads * c];
       const uint32_t kq[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        if ((nib >> e) & 1u) {
-          if (s < kCap) cand[s] = make_uint2(kq[e], static_cast<uint32_t>(lo + 4 * g + e));
-          ++s;
-        }
+        mabove |= (kq[e] > hi1 ? 1u : 0u) << (4 * c + e);
+        mcand |= (kq[e] >= lo1 && kq[e] <= hi1 ? 1u : 0u) << (4 * c + e);
       }
     }
-    if (C > 1) {
-      __syncthreads();
-      const uint32_t tot_c = offs[kMaxCluster], own = offs[rank];
-      for (uint32_t x = tid; x < tot_c && own + x < kCap; x += kThreads) {
-        const uint2 v = cand[own + x];
+    const uint32_t above = __popc(mabove);
+    nc = __popc(mcand);
+    {
+      // This CTA's list: reserve room in every CTA's buffer, write it into the own buffer, then
+      // copy it to the peers.
+      const uint2 ex = block_exclusive2(nc, above, red);
+      if (tid == kThreads - 1) {
+        const uint32_t tot_c = ex.x + nc, tot_a = ex.y + above;
+        uint32_t o[C];  // every reservation in flight before the first result is used
 #pragma unroll
-        for (int r = 0; r < C; ++r)
-          if (static_cast<uint32_t>(r) != rank && offs[r] + x < kCap) st_peer_v2(&cand[offs[r] + x], r, v.x, v.y);
+        for (int r = 0; r < C; ++r) o[r] = (C > 1) ? atom_add_peer(&n_cand, r, tot_c) : atomicAdd(&n_cand, tot_c);
+#pragma unroll
+        for (int r = 0; r < C; ++r) {
+          if (C > 1)
+            st_peer_u32(&above_of[rank], r, tot_a);
+          else
+            above_of[0] = tot_a;
+        }
+#pragma unroll
+        for (int r = 0; r < C; ++r) offs[r] = o[r];
+        offs[kMaxCluster] = tot_c;
+      }
+      __syncthreads();
+      cbase = offs[rank] + ex.x;
+      uint32_t s = cbase;
+      for (uint32_t cm = mcand; cm != 0u;) {  // only the chunks holding candidates
+        const int c = (__ffs(cm) - 1) >> 2;
+        const uint32_t nib = (cm >> (4 * c)) & 0xFu;
+        cm &= ~(0xFu << (4 * c));
+        const int g = tid + kThreads * c;
+        const uint4 q = stk[g];
+        const uint32_t kq[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          if ((nib >> e) & 1u) {
+            if (s < kCap) cand[s] = make_uint2(kq[e], static_cast<uint32_t>(lo + 4 * g + e));
+            ++s;
+          }
+        }
+      }
+      if (C > 1) {
+        __syncthreads();
+        const uint32_t tot_c = offs[kMaxCluster], own = offs[rank];
+        for (uint32_t x = tid; x < tot_c && own + x < kCap; x += kThreads) {
+          const uint2 v = cand[own + x];
+#pragma unroll
+          for (int r = 0; r < C; ++r)
+            if (static_cast<uint32_t>(r) != rank && offs[r] + x < kCap) st_peer_v2(&cand[offs[r] + x], r, v.x, v.y);
+        }
       }
     }
   }
@@ -385,7 +389,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   uint32_t T, r_ties, gt_before, eq_before;
   const uint32_t n_c = n_cand;
-  if (n_c <= kCap) {
+  if (C > 1 && n_c <= kCap) {
     // ---- digits 2 and 3 on the candidates, which every CTA holds in full
     for (uint32_t c = tid; c < n_c; c += kThreads) atomicAdd(&hist[1][(cand[c].x >> 10) & 2047u], 1u);
     hist[0][tid] = 0u;  // the peers finished reading it before the barrier above
