@@ -83,6 +83,14 @@ constexpr int kBarRed0 = 3;  // p sweep partial sums
 constexpr int kBarFin = 5;   // final normaliser of both groups
 static_assert(kSmemBytes <= 232448, "shared memory");
 static_assert(kKvStage % 1024 == 0, "stage alignment (128B-swizzle atoms)");
+// Epilogue tiles in the gather ring (idle once the last PV is done, without a p sweep): rows of
+// one head, padded by 16 bytes so that a warp writing one chunk of each of 32 rows is free of
+// bank conflicts, then copied to HBM by whole rows (coalesced).
+constexpr int kPitchF = kDvCta * 4 + 16;   // fp32 row (a partial O exported between splits)
+constexpr int kPitchB = kDvCta * 2 + 16;   // bf16 row (the output)
+constexpr int kOffOutTile = 64 * kPitchF;  // the combined output tile, after the import tile
+static_assert(128 * kPitchB <= kStages * kKvStage && kOffOutTile + 64 * kPitchB <= kStages * kKvStage,
+              "epilogue tiles fit in the gather ring");
 // This CTA's Q slice (128 head rows x 288 dims) is staged by TMA in gather stages 1.. before the
 // first gathers need them: four 64-dim boxes (SW128) and the 32 rope dims (SW64).
 constexpr int kQBox = 128 * 128;
@@ -456,6 +464,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // exports the other heads' normalised partial O and lse for the other split's CTA.
     const bool own_head = (h >> 6) == split;
     float own_inv_l = 0.f;
+    // the epilogue goes through shared-memory tiles when the gather ring is idle by then
+    const bool staged = p.fuse2 || (p.n_split == 1 && p.p_sel == nullptr);
+    const size_t rows_h = static_cast<size_t>(p.B) * p.Lq * p.H;
     float r = -INFINITY;  // reference of this group's previous block; l is relative to it
     float l = 0.f;
     float lse2 = -INFINITY;
@@ -483,6 +494,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       own_inv_l = inv_l;
       const uint32_t o_cols = static_cast<uint32_t>(wg * (kDvCta / 2));
       if (p.fuse2 && own_head) return;  // finalised after the cluster barrier, from tensor memory
+      // staged: this thread's row goes to an epilogue tile (copied out by whole rows below)
+      uint8_t* trow = p.fuse2 ? sKV + (h & 63) * kPitchF + wg * (kDvCta / 2) * 4
+                              : sKV + h * kPitchB + wg * (kDvCta / 2) * 2;
 #pragma unroll 1
       for (int c0 = 0; c0 < kDvCta / 2; c0 += 16) {
         uint32_t o[16];
@@ -490,7 +504,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld_wait();
         if (!head_ok) continue;
         const int col = static_cast<int>(rank) * kDvCta + static_cast<int>(o_cols) + c0;
-        if (p.n_split == 1 && !p.fuse2) {
+        if (staged && !p.fuse2) {
+          uint4* dst = reinterpret_cast<uint4*>(trow + c0 * 2);
+          dst[0] = make_uint4(pack_bf16x2(__uint_as_float(o[0]) * inv_l, __uint_as_float(o[1]) * inv_l),
+                              pack_bf16x2(__uint_as_float(o[2]) * inv_l, __uint_as_float(o[3]) * inv_l),
+                              pack_bf16x2(__uint_as_float(o[4]) * inv_l, __uint_as_float(o[5]) * inv_l),
+                              pack_bf16x2(__uint_as_float(o[6]) * inv_l, __uint_as_float(o[7]) * inv_l));
+          dst[1] = make_uint4(pack_bf16x2(__uint_as_float(o[8]) * inv_l, __uint_as_float(o[9]) * inv_l),
+                              pack_bf16x2(__uint_as_float(o[10]) * inv_l, __uint_as_float(o[11]) * inv_l),
+                              pack_bf16x2(__uint_as_float(o[12]) * inv_l, __uint_as_float(o[13]) * inv_l),
+                              pack_bf16x2(__uint_as_float(o[14]) * inv_l, __uint_as_float(o[15]) * inv_l));
+        } else if (p.fuse2) {
+          float4* dst = reinterpret_cast<float4*>(trow + c0 * 4);
+#pragma unroll
+          for (int c = 0; c < 16; c += 4)
+            dst[c / 4] = make_float4(__uint_as_float(o[c]) * inv_l, __uint_as_float(o[c + 1]) * inv_l,
+                                     __uint_as_float(o[c + 2]) * inv_l, __uint_as_float(o[c + 3]) * inv_l);
+        } else if (p.n_split == 1) {
           uint4 w0, w1;
           w0.x = pack_bf16x2(__uint_as_float(o[0]) * inv_l, __uint_as_float(o[1]) * inv_l);
           w0.y = pack_bf16x2(__uint_as_float(o[2]) * inv_l, __uint_as_float(o[3]) * inv_l);
@@ -629,6 +659,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     if (!fin) finish();
+    if (staged) {  // the staged rows to HBM, whole rows per warp
+      named_bar_sync(kBarFin, kSoftmaxThreads);
+      if (nblk > 0) {
+        if (p.fuse2) {
+          const int hb = 64 * (split ^ 1);  // the heads this CTA exports
+          const int nrows = max(0, min(64, p.H - hb));
+          float* dst0 = p.part_o + (static_cast<size_t>(split) * rows_h + static_cast<size_t>(row) * p.H + hb) * kDV +
+                        static_cast<int>(rank) * kDvCta;
+          for (int f = threadIdx.x; f < nrows * (kDvCta / 4); f += kSoftmaxThreads) {
+            const int r2 = f / (kDvCta / 4), c = f % (kDvCta / 4);
+            *reinterpret_cast<float4*>(dst0 + static_cast<size_t>(r2) * kDV + 4 * c) =
+                *reinterpret_cast<const float4*>(sKV + r2 * kPitchF + 16 * c);
+          }
+        } else {
+          __nv_bfloat16* dst0 = p.out + static_cast<size_t>(row) * p.H * kDV + static_cast<int>(rank) * kDvCta;
+          for (int f = threadIdx.x; f < p.H * (kDvCta / 8); f += kSoftmaxThreads) {
+            const int r2 = f / (kDvCta / 8), c = f % (kDvCta / 8);
+            *reinterpret_cast<uint4*>(dst0 + static_cast<size_t>(r2) * kDV + 8 * c) =
+                *reinterpret_cast<const uint4*>(sKV + r2 * kPitchB + 16 * c);
+          }
+        }
+      }
+    }
 
     // p emission: slots past the effective length are empty (p = 0)
     if (p.p_sel != nullptr && rank == 0) {
@@ -659,8 +712,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       cluster_barrier();
+      // the other split's export of this CTA's heads into the import tile, whole rows per warp
+      const int hb = 64 * split;
+      const int nrows = max(0, min(64, p.H - hb));
+      {
+        const float* src0 = p.part_o + (static_cast<size_t>(split ^ 1) * rows_h + static_cast<size_t>(row) * p.H + hb) * kDV +
+                            static_cast<int>(rank) * kDvCta;
+        for (int f = threadIdx.x; f < nrows * (kDvCta / 4); f += kSoftmaxThreads) {
+          const int r2 = f / (kDvCta / 4), c = f % (kDvCta / 4);
+          *reinterpret_cast<float4*>(sKV + r2 * kPitchF + 16 * c) =
+              *reinterpret_cast<const float4*>(src0 + static_cast<size_t>(r2) * kDV + 4 * c);
+        }
+      }
+      named_bar_sync(kBarFin, kSoftmaxThreads);
       if (own_head) {  // warp-uniform (a warp covers 32 heads of one 64-head half)
-        const size_t rows_h = static_cast<size_t>(p.B) * p.Lq * p.H;
         const float lse_o = head_ok ? p.part_lse[static_cast<size_t>(split ^ 1) * rows_h + orow] : -INFINITY;
         const float lse_m = (ok && nblk > 0 && head_ok) ? lse2 * kLn2 : -INFINITY;  // natural log
         const float mx = fmaxf(lse_m, lse_o);
@@ -670,7 +735,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float wm = den > 0.f ? em / den * own_inv_l : 0.f;  // own O is not yet normalised
         const float wo = den > 0.f ? eo / den : 0.f;
         const uint32_t o_cols = static_cast<uint32_t>(wg * (kDvCta / 2));
-        const float* other = p.part_o + (static_cast<size_t>(split ^ 1) * rows_h + orow) * kDV;
+        const uint8_t* other = sKV + (h & 63) * kPitchF;                              // import tile row
+        uint8_t* orow_t = sKV + kOffOutTile + (h & 63) * kPitchB + o_cols * 2;  // output tile row
         const bool need_tm = __any_sync(0xFFFFFFFFu, em > 0.f);  // tcgen05.ld is warp-collective
         if (need_tm) tc_fence_after();
 #pragma unroll 1
@@ -683,11 +749,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_ld_wait();
           }
           if (!head_ok) continue;
-          const int col = static_cast<int>(rank) * kDvCta + static_cast<int>(o_cols) + c0;
           float r[16];
 #pragma unroll
           for (int c = 0; c < 16; c += 4) {
-            const float4 u = wo > 0.f ? *reinterpret_cast<const float4*>(other + col + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+            const float4 u = wo > 0.f ? *reinterpret_cast<const float4*>(other + (o_cols + c0 + c) * 4)
+                                      : make_float4(0.f, 0.f, 0.f, 0.f);
             r[c] = fmaf(wo, u.x, em > 0.f ? wm * __uint_as_float(o[c]) : 0.f);
             r[c + 1] = fmaf(wo, u.y, em > 0.f ? wm * __uint_as_float(o[c + 1]) : 0.f);
             r[c + 2] = fmaf(wo, u.z, em > 0.f ? wm * __uint_as_float(o[c + 2]) : 0.f);
@@ -702,11 +768,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           w1.y = pack_bf16x2(r[10], r[11]);
           w1.z = pack_bf16x2(r[12], r[13]);
           w1.w = pack_bf16x2(r[14], r[15]);
-          uint4* dst = reinterpret_cast<uint4*>(p.out + orow * kDV + col);
+          uint4* dst = reinterpret_cast<uint4*>(orow_t + c0 * 2);
           dst[0] = w0;
           dst[1] = w1;
         }
         if (head_ok && rank == 0 && wg == 0 && p.lse) p.lse[orow] = den > 0.f ? mx + logf(den) : -INFINITY;
+      }
+      named_bar_sync(kBarFin, kSoftmaxThreads);
+      __nv_bfloat16* dst0 = p.out + (static_cast<size_t>(row) * p.H + hb) * kDV + static_cast<int>(rank) * kDvCta;
+      for (int f = threadIdx.x; f < nrows * (kDvCta / 8); f += kSoftmaxThreads) {
+        const int r2 = f / (kDvCta / 8), c = f % (kDvCta / 8);
+        *reinterpret_cast<uint4*>(dst0 + static_cast<size_t>(r2) * kDV + 8 * c) =
+            *reinterpret_cast<const uint4*>(sKV + kOffOutTile + r2 * kPitchB + 16 * c);
       }
     }
   }
