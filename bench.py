@@ -385,10 +385,7 @@ def gpu_arm(args, rank, world, device):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "fp8e4m3 indexer, bf16 attention, fp32 accumulate", "data": "synthetic (seeded)",
-        "config": {"workload": wl.name, "B": wl.B, "Lq": wl.Lq, "Lk": wl.Lk, "H_I": wl.H_I,
-                   "d_I": wl.d_I, "k": wl.k, "H": wl.H, "d_qk": wl.d_qk, "d_v": wl.d_v,
-                   "emit_p_and_kl": wl.emit_p, "l2": "flushed (512 MiB write) between steps, outside the step events",
-                   "stage_times": "separate pass with events between launches"},
+        "config": workload_config(wl),
         "e2e": {"value": wl.rows * world / (e2e_ms / 1e3), "unit": "query-tokens/s",
                 "h2d_bytes_per_step": step.h2d_bytes(), "d2h_bytes_per_step": step.d2h_bytes()},
         "gpu_launches": step.launches_per_step * args.steps,
@@ -401,7 +398,14 @@ def gpu_arm(args, rank, world, device):
     return line
 
 
-def reference_arm(args):
+def workload_config(wl):
+    return {"workload": wl.name, "B": wl.B, "Lq": wl.Lq, "Lk": wl.Lk, "H_I": wl.H_I,
+            "d_I": wl.d_I, "k": wl.k, "H": wl.H, "d_qk": wl.d_qk, "d_v": wl.d_v,
+            "emit_p_and_kl": wl.emit_p, "l2": "flushed (512 MiB write) between steps, outside the step events",
+            "stage_times": "separate pass with events between launches"}
+
+
+def reference_arm(args, world):
     wl = dsa_inputs.WORKLOADS[args.workload]
     budget = max(2.0, min(60.0, 20.0 / max(1, args.steps + args.warmup)))
     vals = []
@@ -410,10 +414,11 @@ def reference_arm(args):
         if i >= args.warmup:
             vals.append(v)
     v = statistics.median(vals)
-    return {"metric": METRIC, "value": v, "unit": "query-tokens/s", "n_gpus": 0, "steps": args.steps,
+    # the oracle runs on the host cores of rank 0; n_gpus is the launch's, as on the other arm
+    return {"metric": METRIC, "value": v, "unit": "query-tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": 1e3 * wl.rows / v, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
-            "config": {"workload": wl.name}, "impl": "reference",
+            "config": workload_config(wl), "impl": "reference",
             "cpu_baseline": {"value": v, "unit": "query-tokens/s", "cores": cores, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": v, "unit": "query-tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -432,7 +437,7 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     if args.impl == "reference":
         if rank == 0:
-            print(json.dumps(reference_arm(args)), flush=True)
+            print(json.dumps(reference_arm(args, world)), flush=True)
         return
     local = int(os.environ.get("LOCAL_RANK", "0"))
     device = torch.device("cuda", local)
