@@ -130,7 +130,12 @@ def _mla_case(dsa, wl, idx_np, emit_p=False, check_p=False):
         q_row = dsa_inputs.q_attn(wl, r, 1)[0]
         eo, el, P = ref.sparse_mla_row(q_row, kv[b], idx_np[b, i], wl.d_v, wl.scale, want_P=emit_p)
         parity.check_attention_row(o[b, i], eo, f"row {r}")
-        assert np.abs(l[b, i] - el).max() <= parity.LSE_ATOL, f"lse row {r}"
+        # an empty set has lse = -inf on both sides
+        fin = ~np.isneginf(el)
+        d = np.zeros_like(el)
+        d[fin] = np.abs(l[b, i][fin] - el[fin])
+        d[~fin & ~np.isneginf(l[b, i])] = np.inf
+        assert d.max() <= parity.LSE_ATOL, f"lse row {r}"
         if emit_p:
             parity.check_p_row(ps[b, i], ref.p_sel_row(P, idx_np[b, i]), f"p row {r}")
 
@@ -170,6 +175,21 @@ def test_mla_decode_two_splits_combined_in_kernel(dsa):
     idx[2, 0, 1024:] = -1       # exactly the first split
     idx[3, 0, 40:2000] = -1     # a few entries at both ends
     idx[4, 0, :2047] = -1       # a single valid slot, in the second split
+    _mla_case(dsa, wl, idx)
+
+
+def test_mla_staged_epilogue_fewer_heads(dsa):
+    # enough rows for one CTA pair per row (no KV split) and no p emission: the output rows go
+    # through the shared-memory tile and are written by whole rows; H = 40 leaves most of the
+    # tile's rows unused, and some rows have an empty or a one-entry set
+    wl = dsa_inputs.custom("mla_staged_h40", 29, 2, 40, 600, 64, 128, 16, 256, 40, 576, 512,
+                           1 / math.sqrt(192))
+    rng = np.random.default_rng(31)
+    idx = np.stack([np.stack([rng.permutation(600)[:256] for _ in range(40)]) for _ in range(2)])
+    idx = idx.astype(np.int32)
+    idx[0, 5, :] = -1          # no valid entry
+    idx[1, 7, 1:] = -1         # a single entry
+    idx[1, 9, 100:] = -1       # a ragged tail
     _mla_case(dsa, wl, idx)
 
 
