@@ -26,6 +26,7 @@ import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
 import dsa_inputs  # noqa: E402
+from sparse_attention_tcgen05_b200.sharding import max_over_ranks  # noqa: E402
 
 METRIC = "query-tokens/s (indexer+top-k+sparse MLA) at 1 B200; % of roofline per stage"
 L2_FLUSH_BYTES = 512 << 20
@@ -327,11 +328,7 @@ def gpu_arm(args, rank, world, device):
         stage_ms["topk"].append(e[1].elapsed_time(e[2]))
         stage_ms["sparse_mla"].append(e[2].elapsed_time(e[3]))
         stage_ms["indexer_kl"].append(e[3].elapsed_time(e[4]))
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = t.item()
+    total_ms = max_over_ranks(sum(step_ms), device)  # the slowest rank's time
     ms_per_step = total_ms / args.steps
     qtok = wl.rows * world / (ms_per_step / 1e3)
 
@@ -347,11 +344,7 @@ def gpu_arm(args, rank, world, device):
         step.run_e2e()
     e1.record()
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = t.item()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, device)
 
     work = algorithmic(wl)
     stages = {}
