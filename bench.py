@@ -72,16 +72,26 @@ def algorithmic(wl):
     return {"indexer": ix, "topk": tk, "sparse_mla": ml, "indexer_kl": kl}
 
 
+def _code_only(text: str) -> str:
+    """C/C++/CUDA source with comments removed and whitespace runs collapsed."""
+    import re
+
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
 def source_hash():
-    """Hash of the CUDA sources and the C header: DRAM traffic recorded under profiles/ is
-    reported only while the kernels it was measured on are unchanged."""
+    """Hash of the code (comments and layout ignored) of the CUDA sources and the C header:
+    DRAM traffic recorded under profiles/ is reported only while the kernels it was measured on
+    are unchanged."""
     import hashlib
 
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "sparse_attention_tcgen05_b200", "csrc")
     for name in sorted(os.listdir(csrc)) + ["../../include/dsa.h"]:
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode() + b"\0" + f.read())
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
+            h.update(name.encode() + b"\0" + _code_only(f.read()).encode())
     return h.hexdigest()[:12]
 
 

@@ -15,9 +15,9 @@
 //
 // Tensor memory (512 columns): O [0, 256) fp32, S 2 x 32 fp32 [256, 320), this CTA's slice of
 // Q, 128 heads x 288 bf16, as the A operand of S = Q K^T [320, 464), and P 2 x 16 [464, 496)
-// (bf16, the A operand of O += P V).  Keeping Q in
-// tensor memory means a 32-wide S block only streams its 18 KB gathered tile from shared
-// memory, and frees shared memory for an 8-deep gather ring.
+// (bf16, the A operand of O += P V).  Keeping Q in tensor memory means S only streams the
+// gathered tile (36 KB per pair of blocks) from shared memory, and leaves shared memory to
+// the 3-stage gather ring and the partial-S exchange buffers.
 //
 // Pipeline (per CTA, blocks of 32 selected entries; a p sweep revisits every block):
 //   gather warps   TMA tile::gather4: 4 selected rows per instruction, landing in the
