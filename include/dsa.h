@@ -110,7 +110,7 @@ dsa_status dsa_topk(const float* scores, int32_t* idx, int B, int Lq, int Lk, in
  *   q_bf16  [B, Lq, H, d_qk] bf16     kv_bf16 [B, Lk, d_qk] bf16    idx [B, Lq, k] int32
  *   out_bf16 [B, Lq, H, d_v] bf16     lse [B, Lq, H] fp32 (nullable)
  *   p_sel   [B, Lq, k] fp32 (nullable)
- * Every valid idx must lie in [0, Lk); each row needs at least one valid slot.
+ * Every valid idx must lie in [0, Lk); a row with no valid slot gets out = 0, lse = -infinity.
  * bf16 tensor-core products with fp32 accumulation and fp32 softmax; bf16 output (RNE).
  * Supported: H <= 128, (d_qk, d_v) in {(576, 512), (80, 64)}, 1 <= k <= 65536.
  * ws: dsa_workspace_bytes(DSA_OP_SPARSE_MLA_FWD, B, Lq, Lk, k, H) bytes (split-KV partials
