@@ -58,3 +58,18 @@ def test_workspace_sizes(lib):
     # decode: few rows -> split-KV partials need scratch; prefill: none
     assert dsa.dsa_workspace_bytes(dsa.DSA_OP_SPARSE_MLA_FWD, 32, 1, 32768, 2048, 128) > 0
     assert dsa.dsa_workspace_bytes(dsa.DSA_OP_SPARSE_MLA_FWD, 1, 16384, 16384, 2048, 128) == 0
+
+
+def test_traffic_hash_ignores_comments_but_not_code():
+    import importlib.util
+    import os
+
+    spec = importlib.util.spec_from_file_location(
+        "bench", os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "bench.py"))
+    bench = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(bench)
+    src = "int a = 1; // one\n/* block\n comment */ int b = a + 2;\n"
+    same = "int a = 1;\n\n   int b = a + 2; // other words\n"
+    changed = "int a = 1; int b = a + 3;\n"
+    assert bench._code_only(src) == bench._code_only(same)
+    assert bench._code_only(src) != bench._code_only(changed)
