@@ -3,17 +3,35 @@ top-k -> sparse MLA (and, for the sparse-stage workload, p emission + indexer KL
 batch of seeded synthetic inputs, plus each stage's roofline fraction.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl dsa|reference]
+                  [--scaling weak|strong] [--no-extra] [--peaks] [--dry-run]
 
-N > 1 runs under torchrun, one rank per GPU; every rank processes its own batch of the same
-workload (weak scaling, no data-path collective) and the step time is the max over ranks.
+Default workload: long_prefill_32k (B=1, L=32768 causal, the largest single-GPU workload). With
+N = 1 the same JSON line also carries a benchmark spec block (the 128K-context decode, B=32 queries
+against 131072 keys each) and a `workloads` block with every other workload, each timed the same
+way with fewer steps.
+
+N > 1: `--gpus N` re-launches itself under torch.distributed.run, one rank per GPU (NCCL).
+  weak (default): the job is N copies of the workload's batch (N*B sequences drawn from the
+    seeded streams); each rank takes its sequences with shard_rows, so per-GPU work is fixed.
+  strong: the workload's batch is fixed; decode rows are split with shard_rows and causal
+    prefill rows with shard_causal_rows (rank r computes query rows [start, stop) against keys
+    [0, stop)).
+The sparse-stage loss is summed over ranks (one NCCL all-reduce per step, the path's only
+collective); step time is the max over ranks.  `--dry-run` stops before CUDA: every rank (gloo)
+reports its shard and rank 0 prints them, so the launcher and the sharding are testable on CPU.
+
 `--impl reference` times the fp64 CPU oracle on a bounded sample of the same workload.
+`--peaks` measures the FP8 and bf16 dense GEMM peaks (torch._scaled_mm / torch.matmul, 8192^3)
+and a read-only HBM reference (torch.sum over 1 GiB and 4 GiB) with CUDA events.
 Prints ONE JSON line on rank 0.
 """
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import os
+import socket
 import statistics
 import subprocess
 import sys
@@ -26,10 +44,15 @@ import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
 import dsa_inputs  # noqa: E402
-from sparse_attention_tcgen05_b200.sharding import max_over_ranks  # noqa: E402
+from sparse_attention_tcgen05_b200.sharding import (MLA_WEIGHT, max_over_ranks,  # noqa: E402
+                                                    shard_causal_rows, shard_rows, sum_over_ranks)
 
 METRIC = "query-tokens/s (indexer+top-k+sparse MLA) at 1 B200; % of roofline per stage"
+DEFAULT_WORKLOAD = "long_prefill_32k"
+NORTH_STAR = "decode_128k"
 L2_FLUSH_BYTES = 512 << 20
+# FP8 e4m3 dense rate relative to bf16 (NVIDIA B200 datasheet, dense: 4.5 vs 2.25 PFLOP/s)
+FP8_OVER_BF16 = 2.0
 
 
 def load_peaks():
@@ -112,16 +135,21 @@ def measured_traffic(workload, kernel):
     return None
 
 
-def roofline_us(stage, work, peaks):
-    """Lower-bound time: slower of tensor time (FP8 at 2x the measured bf16 dense peak for the
-    indexer, bf16 for attention) and HBM time at the measured copy bandwidth."""
-    hbm_us = work["bytes"] / (peaks["hbm_gbs"] * 1e9) * 1e6
+def tensor_peak(stage, peaks, sustained):
+    """Dense tensor peak (TFLOP/s) of a stage's contraction: bf16 for attention, FP8 (the bf16
+    measurement times the datasheet's FP8/bf16 ratio) for the indexer; None for the rest."""
+    bf16 = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
     if stage == "indexer":
-        tflops = 2 * peaks["bf16_tflops"]
-    elif stage == "sparse_mla":
-        tflops = peaks["bf16_tflops"]
-    else:
-        tflops = None
+        return FP8_OVER_BF16 * bf16
+    if stage == "sparse_mla":
+        return bf16
+    return None
+
+
+def roofline_us(stage, work, peaks, sustained=False):
+    """Lower-bound time: slower of tensor time and HBM time at the measured copy bandwidth."""
+    hbm_us = work["bytes"] / (peaks["hbm_gbs"] * 1e9) * 1e6
+    tflops = tensor_peak(stage, peaks, sustained)
     tc_us = 2 * work["macs"] / (tflops * 1e12) * 1e6 if tflops else 0.0
     return max(hbm_us, tc_us), ("tensor" if tc_us > hbm_us else "hbm")
 
@@ -135,7 +163,7 @@ class ClockSampler:
     def __init__(self, device_id: str):
         self.proc = None
         self.dev = device_id
-        self.path = os.path.join("/tmp", f"dsa_clocks_{os.getpid()}.csv")
+        self.path = os.path.join("/tmp", f"dsa_clocks_{os.getpid()}_{time.monotonic_ns()}.csv")
 
     def __enter__(self):
         try:
@@ -176,6 +204,10 @@ class ClockSampler:
                 for n, v in zip(names, parts[3:7]):
                     if v.lower().startswith("active"):
                         reasons.add(n)
+        try:
+            os.remove(self.path)
+        except OSError:
+            pass
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
@@ -191,25 +223,79 @@ def pci_id(device) -> str:
         return str(device.index or 0)
 
 
+# ---------------------------------------------------------------------------------- sharding
+@dataclasses.dataclass
+class Shard:
+    """This rank's part of a job: the local workload the kernels are called with, and where its
+    inputs sit in the job's seeded streams (sequences `seqs` of the job's workload, query rows
+    [r0, r1) of each, keys [0, local.Lk))."""
+    job: dsa_inputs.Workload     # the whole job (N * B sequences under weak scaling)
+    local: dsa_inputs.Workload   # what this rank's kernels see
+    seqs: list
+    r0: int
+    r1: int
+
+    def describe(self):
+        return {"seqs": [self.seqs[0], self.seqs[-1] + 1] if self.seqs else [0, 0],
+                "rows": [self.r0, self.r1], "Lk": self.local.Lk}
+
+    def global_rows(self):
+        """Flat query rows (b * Lq + i) of the job that this rank computes."""
+        return [b * self.job.Lq + i for b in self.seqs for i in range(self.r0, self.r1)]
+
+    def host_inputs(self):
+        job, loc = self.job, self.local
+        n = self.r1 - self.r0
+        qI = np.concatenate([dsa_inputs.q_index(job, b * job.Lq + self.r0, n) for b in self.seqs])
+        w = np.concatenate([dsa_inputs.w_index(job, b * job.Lq + self.r0, n) for b in self.seqs])
+        q = np.concatenate([dsa_inputs.q_attn(job, b * job.Lq + self.r0, n) for b in self.seqs])
+        kI = np.stack([dsa_inputs.k_index(job, b)[:loc.Lk] for b in self.seqs])
+        kv = np.stack([dsa_inputs.kv_latent(job, b)[:loc.Lk] for b in self.seqs])
+        return {"qI": qI.reshape(loc.B, loc.Lq, loc.H_I, loc.d_I), "kI": kI,
+                "w": w.reshape(loc.B, loc.Lq, loc.H_I), "q": q.reshape(loc.B, loc.Lq, loc.H, loc.d_qk),
+                "kv": kv}
+
+
+def make_shard(wl, rank, world, scaling):
+    if scaling == "weak":
+        job = dataclasses.replace(wl, B=wl.B * world)
+        s0, s1 = shard_rows(job.B, rank, world)
+        return Shard(job, dataclasses.replace(wl, B=s1 - s0), list(range(s0, s1)), 0, wl.Lq)
+    if wl.Lq == 1:  # decode: one query per sequence, split the sequences
+        s0, s1 = shard_rows(wl.B, rank, world)
+        if s1 <= s0:
+            raise SystemExit(f"strong scaling: {world} ranks for {wl.B} decode rows")
+        return Shard(wl, dataclasses.replace(wl, B=s1 - s0), list(range(s0, s1)), 0, 1)
+    # causal prefill: every sequence's query rows [start, stop), balanced by causal work; the
+    # rank sees keys [0, stop + Lk - Lq), so row i of the shard keeps its position t
+    start, stop = shard_causal_rows(wl.Lq, wl.Lk, wl.k, rank, world, mla_weight=MLA_WEIGHT)
+    if stop <= start:
+        raise SystemExit(f"strong scaling: {world} ranks for {wl.Lq} query rows")
+    local = dataclasses.replace(wl, Lq=stop - start, Lk=stop + (wl.Lk - wl.Lq))
+    return Shard(wl, local, list(range(wl.B)), start, stop)
+
+
 # ---------------------------------------------------------------------------------- GPU arm
 class Step:
     """Device buffers and the calls of one step through the C ABI."""
 
-    def __init__(self, wl, device):
+    def __init__(self, shard, device, keep_host=True):
         import sparse_attention_tcgen05_b200 as dsa
 
+        wl = shard.local
         self.dsa, self.wl, self.dev = dsa, wl, device
         B, Lq, Lk = wl.B, wl.Lq, wl.Lk
-        self.h = {  # pinned host copies of the inputs (for the end-to-end measurement)
-            "qI": torch.from_numpy(dsa_inputs.q_index(wl).reshape(B, Lq, wl.H_I, wl.d_I)).view(
-                torch.float8_e4m3fn).pin_memory(),
-            "kI": torch.from_numpy(dsa_inputs.k_index(wl)).view(torch.float8_e4m3fn).pin_memory(),
-            "w": torch.from_numpy(dsa_inputs.w_index(wl).reshape(B, Lq, wl.H_I)).pin_memory(),
-            "q": torch.from_numpy(dsa_inputs.q_attn(wl).view(np.int16).reshape(B, Lq, wl.H, wl.d_qk)).view(
-                torch.bfloat16).pin_memory(),
-            "kv": torch.from_numpy(dsa_inputs.kv_latent(wl).view(np.int16)).view(torch.bfloat16).pin_memory(),
-        }
-        self.d = {k: v.to(device) for k, v in self.h.items()}
+        x = shard.host_inputs()
+        h = {"qI": torch.from_numpy(x["qI"]).view(torch.float8_e4m3fn),
+             "kI": torch.from_numpy(x["kI"]).view(torch.float8_e4m3fn),
+             "w": torch.from_numpy(x["w"]),
+             "q": torch.from_numpy(x["q"].view(np.int16)).view(torch.bfloat16),
+             "kv": torch.from_numpy(x["kv"].view(np.int16)).view(torch.bfloat16)}
+        del x
+        # pinned host copies of the inputs (for the end-to-end measurement)
+        self.h = {k_: v.pin_memory() for k_, v in h.items()} if keep_host else None
+        self.d = {k_: v.to(device) for k_, v in (self.h or h).items()}
+        del h
         self.scores = torch.empty(B, Lq, Lk, dtype=torch.float32, device=device)
         self.idx = torch.empty(B, Lq, wl.k, dtype=torch.int32, device=device)
         self.out = torch.empty(B, Lq, wl.H, wl.d_v, dtype=torch.bfloat16, device=device)
@@ -219,8 +305,11 @@ class Step:
         nws = max(dsa.dsa_workspace_bytes(dsa.DSA_OP_SPARSE_MLA_FWD, B, Lq, Lk, wl.k, wl.H),
                   dsa.dsa_workspace_bytes(dsa.DSA_OP_INDEXER_KL, B, Lq, Lk, wl.k, 0), 16)
         self.ws = torch.empty(nws, dtype=torch.uint8, device=device)
-        self.out_h = torch.empty(self.out.shape, dtype=torch.bfloat16).pin_memory()
-        self.loss_h = torch.empty(1, dtype=torch.float32).pin_memory()
+        if keep_host:
+            self.out_h = torch.empty(self.out.shape, dtype=torch.bfloat16).pin_memory()
+            self.loss_h = torch.empty(1, dtype=torch.float32).pin_memory()
+        self.reduce_loss = wl.emit_p and torch.distributed.is_initialized() and \
+            torch.distributed.get_world_size() > 1
         # the split-KV combine is a separate launch only with more than two splits (two splits
         # combine inside the attention kernel)
         self.launches_per_step = 3 + (2 if wl.emit_p else 0) + (1 if self._mla_splits() > 2 else 0)
@@ -248,6 +337,8 @@ class Step:
             ev[3].record()
         if wl.emit_p:
             dsa.dsa_indexer_kl(self.scores, self.idx, self.p, self.loss, None, self.ws)
+            if self.reduce_loss:
+                sum_over_ranks(self.loss)  # the sharded loss: one all-reduce of 4 bytes
         if ev:
             ev[4].record()
 
@@ -274,7 +365,6 @@ def cpu_oracle_sample(wl, budget_s=12.0, max_rows=None):
     from oracle import oracle as ref
 
     cores = os.cpu_count() or 1
-    rows_all = dsa_inputs.sample_rows(wl, 0) if wl.Lq > 1 else list(range(wl.rows))
     rng = np.random.default_rng(17)
     pool = rng.permutation(wl.rows)
     kI = dsa_inputs.k_index(wl)
@@ -298,26 +388,26 @@ def cpu_oracle_sample(wl, budget_s=12.0, max_rows=None):
     n = min(n, wl.rows)
     rows = [int(x) for x in pool[:n]]
     dt = run(rows)
-    del rows_all
     return len(rows) / dt, cores, f"{len(rows)} of {wl.rows} query rows (seeded uniform), {dt:.1f} s"
 
 
-def gpu_arm(args, rank, world, device):
-    wl = dsa_inputs.WORKLOADS[args.workload]
-    step = Step(wl, device)
-    peaks = load_peaks()
+def measure(shard, device, steps, warmup, world, peaks, e2e=True):
+    """Times `steps` steps of the shard (after `warmup`), each between one pair of CUDA events on
+    the launching stream with an L2 flush before it; returns the per-workload record."""
+    wl = shard.local
+    step = Step(shard, device, keep_host=e2e)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         step.run()
     torch.cuda.synchronize()
     # Timed region: each step's launches go back to back between one pair of events (events
     # between the kernels would stop each launch from overlapping the previous kernel's tail).
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
     with ClockSampler(pci_id(device)) as clk:
-        for i in range(args.steps):
+        for i in range(steps):
             flush.fill_(i & 0xFF)  # evict L2 between steps (outside the step's events)
             evs[i][0].record()
             step.run()
@@ -329,7 +419,7 @@ def gpu_arm(args, rank, world, device):
     # Per-stage times (for the stage roofline fractions) from a separate pass of the same steps
     # with an event between every two launches.
     stage_ms = {"indexer": [], "topk": [], "sparse_mla": [], "indexer_kl": []}
-    for i in range(args.steps):
+    for i in range(steps):
         flush.fill_(i & 0xFF)
         e = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
         step.run(e)
@@ -339,73 +429,124 @@ def gpu_arm(args, rank, world, device):
         stage_ms["sparse_mla"].append(e[2].elapsed_time(e[3]))
         stage_ms["indexer_kl"].append(e[3].elapsed_time(e[4]))
     total_ms = max_over_ranks(sum(step_ms), device)  # the slowest rank's time
-    ms_per_step = total_ms / args.steps
-    qtok = wl.rows * world / (ms_per_step / 1e3)
+    ms_per_step = total_ms / steps
+    rows_all = shard.job.rows if world > 1 else wl.rows  # query rows of all ranks
+    qtok = rows_all / (ms_per_step / 1e3)
 
-    # end-to-end through host buffers
-    e2e_steps = max(2, min(args.steps, 5))
-    step.run_e2e()
-    torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(e2e_steps):
+    rec_e2e = None
+    if e2e:
+        e2e_steps = max(2, min(steps, 5))
         step.run_e2e()
-    e1.record()
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, device)
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(e2e_steps):
+            step.run_e2e()
+        e1.record()
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, device)
+        rec_e2e = {"value": rows_all / (e2e_ms / 1e3), "unit": "query-tokens/s",
+                   "h2d_bytes_per_step": step.h2d_bytes(), "d2h_bytes_per_step": step.d2h_bytes()}
 
+    # prefill steps last tens of milliseconds and repeat back to back: their contractions are
+    # held to the sustained (power-capped) GEMM peak; decode steps last microseconds (burst)
+    sustained = wl.Lq > 1 and ms_per_step >= 5.0
     work = algorithmic(wl)
     stages = {}
     for name, ms in stage_ms.items():
         if name == "indexer_kl" and not wl.emit_p:
             continue
         med = statistics.median(ms)
-        r_us, bound = roofline_us(name, work[name], peaks)
+        r_us, bound = roofline_us(name, work[name], peaks, sustained)
         stages[name] = {"ms": round(med, 4), "roofline_us": round(r_us, 2), "bound": bound,
                         "frac": round(r_us / (med * 1e3), 4),
                         "gbs": round(work[name]["bytes"] / (med * 1e-3) / 1e9, 1),
                         "tflops": round(2 * work[name]["macs"] / (med * 1e-3) / 1e12, 1)}
+        tp = tensor_peak(name, peaks, sustained)
+        if tp:
+            stages[name]["tensor_peak_tflops"] = round(tp, 1)
     path_roof = sum(v["roofline_us"] for v in stages.values())
     dom = max(stages, key=lambda s: stages[s]["ms"])
     ds = stages[dom]
     if ds["bound"] == "hbm":
         roof = {"kernel": dom, "bound": "hbm", "achieved": ds["gbs"], "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": round(ds["gbs"] / peaks["hbm_gbs"], 4)}
+        src = peaks["source"] + " copy bandwidth"
     else:
-        peak_t = peaks["bf16_tflops"] * (2 if dom == "indexer" else 1)
-        roof = {"kernel": dom, "bound": "tensor", "achieved": ds["tflops"], "peak": peak_t,
+        peak_t = tensor_peak(dom, peaks, sustained)
+        roof = {"kernel": dom, "bound": "tensor", "achieved": ds["tflops"], "peak": round(peak_t, 1),
                 "unit": "TFLOP/s", "frac": round(ds["tflops"] / peak_t, 4)}
-    roof["traffic"] = measured_traffic(wl.name, dom)
-    roof["peak_source"] = peaks["source"] + (" (fp8 = 2x measured bf16)" if roof["unit"] == "TFLOP/s" and dom == "indexer" else "")
+        src = f"{peaks['source']} bf16 GEMM, {'sustained' if sustained else 'burst'}" + \
+            (" x2 for fp8 (datasheet ratio)" if dom == "indexer" else "")
+    roof["traffic"] = measured_traffic(wl.name, dom) if world == 1 else None
+    roof["peak_source"] = src
+    return {"workload": wl.name, "rows": rows_all, "steps": steps, "warmup": warmup,
+            "ms_per_step": ms_per_step, "value": qtok, "unit": "query-tokens/s",
+            "path_roofline_us": round(path_roof, 2),
+            "path_roofline_frac": round(path_roof / (ms_per_step * 1e3), 4),
+            "stages": stages, "roofline": roof, "clocks": clk.summary(), "e2e": rec_e2e,
+            "gpu_launches": step.launches_per_step * steps}
+
+
+def workload_config(wl, world=1, scaling="weak", shard=None):
+    cfg = {"workload": wl.name, "B": wl.B, "Lq": wl.Lq, "Lk": wl.Lk, "H_I": wl.H_I,
+           "d_I": wl.d_I, "k": wl.k, "H": wl.H, "d_qk": wl.d_qk, "d_v": wl.d_v,
+           "emit_p_and_kl": wl.emit_p, "l2": "flushed (512 MiB write) between steps, outside the step events",
+           "stage_times": "separate pass with events between launches"}
+    if world > 1:
+        cfg["parallelism"] = f"rows over {world} ranks ({scaling} scaling)"
+        cfg["job_rows"] = shard.job.rows
+    return cfg
+
+
+def gpu_arm(args, rank, world, device):
+    wl = dsa_inputs.WORKLOADS[args.workload]
+    shard = make_shard(wl, rank, world, args.scaling)
+    peaks = load_peaks()
+    rec = measure(shard, device, args.steps, args.warmup, world, peaks, e2e=True)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, cores, sample = cpu_oracle_sample(wl)
         cpu = {"value": v, "unit": "query-tokens/s", "cores": cores, "kind": "oracle", "sample": sample}
     line = {
-        "metric": METRIC, "value": qtok, "unit": "query-tokens/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "metric": METRIC, "value": rec["value"], "unit": "query-tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": rec["ms_per_step"],
+        "higher_is_better": True, "scaling": args.scaling, "vs_baseline": None,
         "dtype": "fp8e4m3 indexer, bf16 attention, fp32 accumulate", "data": "synthetic (seeded)",
-        "config": workload_config(wl),
-        "e2e": {"value": wl.rows * world / (e2e_ms / 1e3), "unit": "query-tokens/s",
-                "h2d_bytes_per_step": step.h2d_bytes(), "d2h_bytes_per_step": step.d2h_bytes()},
-        "gpu_launches": step.launches_per_step * args.steps,
-        "roofline": roof,
-        "stages": stages,
-        "path_roofline_frac": round(path_roof / (ms_per_step * 1e3), 4),
-        "clocks": clk.summary(),
+        "config": workload_config(wl, world, args.scaling, shard),
+        "e2e": rec["e2e"],
+        "gpu_launches": rec["gpu_launches"],
+        "roofline": rec["roofline"],
+        "stages": rec["stages"],
+        "path_roofline_us": rec["path_roofline_us"],
+        "path_roofline_frac": rec["path_roofline_frac"],
+        "clocks": rec["clocks"],
         "cpu_baseline": cpu,
     }
+    if world == 1 and not args.no_extra:
+        # every other workload, timed the same way (fewer steps, no host round trip)
+        extra = {}
+        names = [NORTH_STAR] + [n for n in ("decode_32k", "prefill_2x8k", "indexer_kl_16k", "tiny_prefill")
+                                if n != args.workload]
+        for name in names:
+            if name == args.workload:
+                continue
+            w2 = dsa_inputs.WORKLOADS[name]
+            torch.cuda.empty_cache()
+            r = measure(make_shard(w2, 0, 1, "weak"), device, args.extra_steps, max(3, args.warmup // 2),
+                        1, peaks, e2e=False)
+            r.pop("e2e")
+            r["config"] = workload_config(w2)
+            extra[name] = r
+        if NORTH_STAR in extra:
+            line["north_star"] = extra.pop(NORTH_STAR)
+            line["north_star"]["target"] = "path_roofline_frac >= 0.60"
+        line["workloads"] = extra
+        line["gpu_launches"] += sum(r["gpu_launches"] for r in extra.values()) + \
+            line.get("north_star", {}).get("gpu_launches", 0)
     return line
-
-
-def workload_config(wl):
-    return {"workload": wl.name, "B": wl.B, "Lq": wl.Lq, "Lk": wl.Lk, "H_I": wl.H_I,
-            "d_I": wl.d_I, "k": wl.k, "H": wl.H, "d_qk": wl.d_qk, "d_v": wl.d_v,
-            "emit_p_and_kl": wl.emit_p, "l2": "flushed (512 MiB write) between steps, outside the step events",
-            "stage_times": "separate pass with events between launches"}
 
 
 def reference_arm(args, world):
@@ -420,11 +561,98 @@ def reference_arm(args, world):
     # the oracle runs on the host cores of rank 0; n_gpus is the launch's, as on the other arm
     return {"metric": METRIC, "value": v, "unit": "query-tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": 1e3 * wl.rows / v, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+            "scaling": args.scaling, "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
             "config": workload_config(wl), "impl": "reference",
             "cpu_baseline": {"value": v, "unit": "query-tokens/s", "cores": cores, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": v, "unit": "query-tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+# ---------------------------------------------------------------------------------- peaks
+def peaks_arm(device):
+    """Dense GEMM peaks (FP8 e4m3 via torch._scaled_mm, bf16 via torch.matmul; 8192^3, best of 10)
+    and read-only / copy HBM references (torch.sum over 1 GiB and 4 GiB, copy_ of 1 GiB; best of
+    10), all timed with CUDA events, with the clocks sampled during the loops."""
+    def best(fn, reps=10):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        return min(ts), statistics.median(ts)
+
+    res = {"metric": "measured peaks", "device": torch.cuda.get_device_name(device)}
+    with ClockSampler(pci_id(device)) as clk:
+        n = 8192
+        a = torch.randn(n, n, device=device).to(torch.float8_e4m3fn)
+        bt = torch.randn(n, n, device=device).to(torch.float8_e4m3fn).t()  # column-major B
+        one = torch.ones((), device=device)
+        t, tm = best(lambda: torch._scaled_mm(a, bt, scale_a=one, scale_b=one, out_dtype=torch.bfloat16))
+        res["fp8_e4m3_tflops"] = {"best": 2 * n ** 3 / (t * 1e-3) / 1e12, "median": 2 * n ** 3 / (tm * 1e-3) / 1e12}
+        del a, bt
+        a = torch.randn(n, n, device=device, dtype=torch.bfloat16)
+        b = torch.randn(n, n, device=device, dtype=torch.bfloat16)
+        t, tm = best(lambda: torch.matmul(a, b))
+        res["bf16_tflops"] = {"best": 2 * n ** 3 / (t * 1e-3) / 1e12, "median": 2 * n ** 3 / (tm * 1e-3) / 1e12}
+        del a, b
+        for gib in (1, 4):
+            x = torch.ones(gib << 28, device=device, dtype=torch.float32)
+            t, tm = best(lambda: torch.sum(x))
+            res[f"hbm_read_sum_{gib}gib_gbs"] = {"best": (gib << 30) / (t * 1e-3) / 1e9,
+                                                 "median": (gib << 30) / (tm * 1e-3) / 1e9}
+            del x
+        x = torch.ones(1 << 28, device=device, dtype=torch.float32)
+        y = torch.empty_like(x)
+        t, tm = best(lambda: y.copy_(x))
+        res["hbm_copy_1gib_gbs"] = {"best": 2 * (1 << 30) / (t * 1e-3) / 1e9,
+                                    "median": 2 * (1 << 30) / (tm * 1e-3) / 1e9}
+        torch.cuda.synchronize()
+    res["clocks"] = clk.summary()
+    return res
+
+
+# ---------------------------------------------------------------------------------- launcher
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def relaunch(args):
+    """Re-run this script under torch.distributed.run with one rank per GPU."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={args.gpus}",
+           "--master-addr", "127.0.0.1", "--master-port", str(_free_port()), os.path.abspath(__file__),
+           *sys.argv[1:]]
+    return subprocess.call(cmd)
+
+
+def dry_run(args, rank, world):
+    """The launch and the sharding without CUDA: every rank reports its shard over gloo."""
+    import datetime
+
+    if world > 1:
+        torch.distributed.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+    wl = dsa_inputs.WORKLOADS[args.workload]
+    sh = make_shard(wl, rank, world, args.scaling)
+    mine = {"rank": rank, **sh.describe(), "global_rows": [min(sh.global_rows()), max(sh.global_rows()) + 1],
+            "n_rows": len(sh.global_rows())}
+    allv = [None] * world
+    if world > 1:
+        torch.distributed.all_gather_object(allv, mine)
+    else:
+        allv = [mine]
+    if rank == 0:
+        print(json.dumps({"dry_run": True, "n_gpus": world, "scaling": args.scaling, "workload": wl.name,
+                          "job_rows": sh.job.rows, "shards": allv}), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
 
 
 def main():
@@ -432,12 +660,26 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="decode_32k", choices=sorted(dsa_inputs.WORKLOADS))
+    ap.add_argument("--extra-steps", type=int, default=8, help="timed steps of each non-headline workload")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(dsa_inputs.WORKLOADS))
     ap.add_argument("--impl", default="dsa", choices=["dsa", "reference"])
+    ap.add_argument("--scaling", default="weak", choices=["weak", "strong"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true", help="time the headline workload only")
+    ap.add_argument("--peaks", action="store_true", help="measure GEMM and HBM peaks instead")
+    ap.add_argument("--dry-run", action="store_true", help="launch and shard without CUDA")
     args = ap.parse_args()
+    if args.warmup < 3 and not args.dry_run:
+        ap.error("--warmup must be at least 3")
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        sys.exit(relaunch(args))
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
+    if world != args.gpus:
+        sys.exit(f"--gpus {args.gpus} but WORLD_SIZE {world}")
+    if args.dry_run:
+        dry_run(args, rank, world)
+        return
     if args.impl == "reference":
         if rank == 0:
             print(json.dumps(reference_arm(args, world)), flush=True)
@@ -445,6 +687,10 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
+    if args.peaks:
+        if rank == 0:
+            print(json.dumps(peaks_arm(device)), flush=True)
+        return
     if world > 1:
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),

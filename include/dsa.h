@@ -153,12 +153,36 @@ dsa_status dsa_indexer_kl(const float* scores, const int32_t* idx, const float* 
  *   - Every call shares the one array and leaves its rows in it; each call writes every row
  *     it reads, so nothing needs clearing, but calls whose kernels overlap on the GPU (on
  *     different streams, or from different host threads) race on it.  Serialise them.
- *   - No cudaMalloc, cudaFree or other allocating routine is called.
- * Results are identical to dsa_indexer_kl on the same inputs.
+ *   - No cudaMalloc, cudaFree or other allocating routine is called.  CUDA itself places the
+ *     library's device code, this array included, in a device's memory when the library first
+ *     launches a kernel or looks the array up on that device (already at load time under
+ *     CUDA_MODULE_LOADING=EAGER).  A caller that will reserve all free device memory should
+ *     therefore make one call of this entry point on each device before it does so.
+ * Results are bit-identical to dsa_indexer_kl on the same inputs (same kernels, same
+ * fixed-order sum).  Bad pointers, sizes or alignment (loss_per_query included) return
+ * DSA_ERR_INVALID_ARG before anything is launched.
  */
 dsa_status dsa_indexer_kl_noalloc(const float* scores, const int32_t* idx, const float* p_sel,
                                   int B, int Lq, int Lk, int k, float* loss,
                                   float* loss_per_query, dsa_stream_t stream);
+
+/*
+ * Failure detection ("DeepSeek-V3.2" analysis page, sec. 5.1: check inputs at entry and keep the
+ * system observable).  Every wait inside a kernel of this library is bounded; by default a wait
+ * gives up after 2 s, records DSA_ERR_TIMEOUT in the device status word and lets its kernel
+ * return.  dsa_set_wait_limit_ns sets that bound, in nanoseconds, for kernels launched
+ * afterwards on the CURRENT device (0 restores the default).  It is a synchronous copy: call it
+ * while no kernel of this library runs on the device.
+ */
+dsa_status dsa_set_wait_limit_ns(uint64_t ns);
+
+/*
+ * Diagnostic: launches one warp on `stream` that waits on an mbarrier nothing arrives on.  The
+ * wait expires after the current limit, DSA_ERR_TIMEOUT is recorded (read it with
+ * dsa_last_device_status) and the kernel returns; the context stays usable.  Lets a test check
+ * the failure-detection path without any fault.
+ */
+dsa_status dsa_selftest_wait(dsa_stream_t stream);
 
 /*
  * Waits for `stream`, then returns and clears the device status word that kernels set

@@ -18,14 +18,14 @@ from . import build as _build
 __all__ = [
     "DsaError", "load", "dsa_status_str", "dsa_version", "dsa_workspace_bytes", "dsa_indexer",
     "dsa_topk", "dsa_sparse_mla_fwd", "dsa_indexer_kl", "dsa_indexer_kl_noalloc",
-    "dsa_last_device_status",
+    "dsa_last_device_status", "dsa_set_wait_limit_ns", "dsa_selftest_wait",
     "DSA_OP_INDEXER", "DSA_OP_TOPK", "DSA_OP_SPARSE_MLA_FWD", "DSA_OP_INDEXER_KL", "EXPORTED",
 ]
 
 DSA_OP_INDEXER, DSA_OP_TOPK, DSA_OP_SPARSE_MLA_FWD, DSA_OP_INDEXER_KL = 0, 1, 2, 3
 EXPORTED = ("dsa_status_str", "dsa_version", "dsa_workspace_bytes", "dsa_indexer", "dsa_topk",
             "dsa_sparse_mla_fwd", "dsa_indexer_kl", "dsa_indexer_kl_noalloc",
-            "dsa_last_device_status")
+            "dsa_last_device_status", "dsa_set_wait_limit_ns", "dsa_selftest_wait")
 
 
 class DsaError(RuntimeError):
@@ -58,8 +58,11 @@ def load(rebuild: bool = False) -> ctypes.CDLL:
         lib.dsa_indexer_kl.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, vp, vp, sz, vp]
         lib.dsa_indexer_kl_noalloc.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, vp, vp]
         lib.dsa_last_device_status.argtypes = [vp]
+        lib.dsa_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+        lib.dsa_selftest_wait.argtypes = [vp]
         for name in ("dsa_indexer", "dsa_topk", "dsa_sparse_mla_fwd", "dsa_indexer_kl",
-                     "dsa_indexer_kl_noalloc", "dsa_last_device_status"):
+                     "dsa_indexer_kl_noalloc", "dsa_last_device_status", "dsa_set_wait_limit_ns",
+                     "dsa_selftest_wait"):
             getattr(lib, name).restype = i32
         _lib = lib
     return _lib
@@ -197,6 +200,18 @@ def dsa_indexer_kl_noalloc(scores: torch.Tensor, idx: torch.Tensor, p_sel: torch
     _raise("dsa_indexer_kl_noalloc",
            load().dsa_indexer_kl_noalloc(_ptr(scores), _ptr(idx), _ptr(p_sel), B, Lq, Lk, k,
                                          _ptr(loss), _ptr(loss_per_query), _stream(stream)))
+
+
+def dsa_set_wait_limit_ns(ns: int) -> None:
+    """Bound (ns) of every in-kernel wait for kernels launched afterwards on the current device;
+    0 restores the default of 2 s."""
+    _raise("dsa_set_wait_limit_ns", load().dsa_set_wait_limit_ns(int(ns)))
+
+
+def dsa_selftest_wait(stream=None) -> None:
+    """Launch one warp that waits on an mbarrier nothing arrives on (it gives up after the wait
+    limit and records DSA_ERR_TIMEOUT)."""
+    _raise("dsa_selftest_wait", load().dsa_selftest_wait(_stream(stream)))
 
 
 def dsa_last_device_status(stream=None) -> int:

@@ -7,6 +7,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 #include <utility>
 
@@ -31,22 +32,29 @@ struct DeviceInfo {
 };
 
 constexpr int kMaxDevices = 64;
+// Per-device facts, looked up once and cached only when the lookup succeeded (a failed lookup,
+// e.g. before the context is ready, is retried on the next call).
 DeviceInfo g_dev[kMaxDevices];
-std::once_flag g_dev_once[kMaxDevices];
+std::atomic<bool> g_dev_ok[kMaxDevices];
+std::mutex g_mu;
 
 dsa_status current_device(DeviceInfo& out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DSA_ERR_CUDA;
-  std::call_once(g_dev_once[dev], [dev]() {
-    int major = 0, minor = 0, sms = 0;
-    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return;
-    if (cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) return;
-    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return;
-    g_dev[dev].sm100 = (major == 10 && minor == 0);
-    g_dev[dev].sms = sms;
-    g_dev[dev].ok = true;
-  });
-  if (!g_dev[dev].ok) return DSA_ERR_CUDA;
+  if (!g_dev_ok[dev].load(std::memory_order_acquire)) {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!g_dev_ok[dev].load(std::memory_order_relaxed)) {
+      int major = 0, minor = 0, sms = 0;
+      if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+          cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+          cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return DSA_ERR_CUDA;
+      g_dev[dev].sm100 = (major == 10 && minor == 0);
+      g_dev[dev].sms = sms;
+      g_dev[dev].ok = true;
+      g_dev_ok[dev].store(true, std::memory_order_release);
+    }
+  }
   if (!g_dev[dev].sm100) return DSA_ERR_NO_SM100;
   out = g_dev[dev];
   return DSA_OK;
@@ -65,16 +73,17 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 EncodeTiledFn get_encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, []() {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  });
-  return fn;
+  static std::atomic<EncodeTiledFn> cached{nullptr};
+  EncodeTiledFn fn = cached.load(std::memory_order_acquire);
+  if (fn) return fn;
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+      q == cudaDriverEntryPointSuccess) {
+    fn = reinterpret_cast<EncodeTiledFn>(p);
+    cached.store(fn, std::memory_order_release);
+  }
+  return fn;  // nullptr: looked up again on the next call
 }
 
 // 2-D row-major tensor [outer, inner] with `row_bytes` between rows; box [box_outer, box_inner].
@@ -313,27 +322,44 @@ dsa_status launch_mla(const void* q, const void* kv, const int32_t* idx, int B, 
 constexpr int kKlNoAllocMaxRows = 1 << 20;  // 4 MiB of fp32 per device
 static __device__ __align__(256) float g_kl_rows_scratch[kKlNoAllocMaxRows];
 
-struct KlScratch {
-  std::once_flag once;
-  float* ptr = nullptr;
-  cudaError_t err = cudaSuccess;
-};
-KlScratch g_kl_scratch[kMaxDevices];
+float* g_kl_scratch_ptr[kMaxDevices];
+std::atomic<bool> g_kl_scratch_ok[kMaxDevices];
 
 // Device address of g_kl_rows_scratch on the current device.  The name itself is only a host
-// stand-in, so the address must come from cudaGetSymbolAddress with that device current.
+// stand-in, so the address must come from cudaGetSymbolAddress with that device current.  Only a
+// successful lookup is cached; a failed one is retried on the next call.
 dsa_status kl_scratch_for_current_device(float** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DSA_ERR_CUDA;
-  KlScratch& s = g_kl_scratch[dev];
-  std::call_once(s.once, [&s]() {
-    void* p = nullptr;
-    s.err = cudaGetSymbolAddress(&p, g_kl_rows_scratch);
-    s.ptr = static_cast<float*>(p);
-  });
-  if (s.err != cudaSuccess || s.ptr == nullptr) return DSA_ERR_CUDA;
-  *out = s.ptr;
+  if (!g_kl_scratch_ok[dev].load(std::memory_order_acquire)) {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!g_kl_scratch_ok[dev].load(std::memory_order_relaxed)) {
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_kl_rows_scratch) != cudaSuccess || p == nullptr) {
+        cudaGetLastError();  // clear the (non-sticky) error so that the next call starts clean
+        return DSA_ERR_CUDA;
+      }
+      g_kl_scratch_ptr[dev] = static_cast<float*>(p);
+      g_kl_scratch_ok[dev].store(true, std::memory_order_release);
+    }
+  }
+  *out = g_kl_scratch_ptr[dev];
   return DSA_OK;
+}
+
+// ------------------------------------------------------------------------------ wait self-test
+// One warp waits on an mbarrier that nothing arrives on: the bounded wait gives up after the
+// limit in force and records DSA_ERR_TIMEOUT (site 90), and the kernel returns.
+__global__ void wait_selftest_kernel() {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    dsa::mbar_init(&bar, 1);
+    abort_flag = 0;
+    dsa::fence_barrier_init();
+  }
+  __syncwarp();
+  dsa::mbar_wait(&bar, 0, &abort_flag, 90);
 }
 
 }  // namespace
@@ -353,7 +379,7 @@ const char* dsa_status_str(dsa_status s) {
   return "DSA_ERR_UNKNOWN";
 }
 
-int dsa_version(void) { return 100; }
+int dsa_version(void) { return 101; }
 
 size_t dsa_workspace_bytes(int op, int B, int Lq, int Lk, int k, int H) {
   (void)Lk;
@@ -456,13 +482,15 @@ dsa_status dsa_indexer_kl(const float* scores, const int32_t* idx, const float* 
                           size_t ws_bytes, dsa_stream_t stream) {
   if (!scores || !idx || !p_sel || !loss) return DSA_ERR_INVALID_ARG;
   if (B <= 0 || Lq <= 0 || Lk <= 0 || Lq > Lk || k <= 0) return DSA_ERR_INVALID_ARG;
-  if (!aligned16(scores) || !aligned16(idx) || !aligned16(p_sel) || (reinterpret_cast<uintptr_t>(loss) & 3u))
+  if (!aligned16(scores) || !aligned16(idx) || !aligned16(p_sel) || (reinterpret_cast<uintptr_t>(loss) & 3u) ||
+      (loss_per_query && !aligned16(loss_per_query)))
     return DSA_ERR_INVALID_ARG;
   const long rows = static_cast<long>(B) * Lq;
   if (rows > INT32_MAX) return DSA_ERR_UNSUPPORTED;
   float* per_row = loss_per_query;
   if (per_row == nullptr) {
-    if (ws == nullptr || ws_bytes < static_cast<size_t>(rows) * sizeof(float)) return DSA_ERR_INVALID_ARG;
+    if (ws == nullptr || ws_bytes < static_cast<size_t>(rows) * sizeof(float) || !aligned16(ws))
+      return DSA_ERR_INVALID_ARG;
     per_row = static_cast<float*>(ws);
   }
   DeviceInfo dev;
@@ -481,7 +509,8 @@ dsa_status dsa_indexer_kl_noalloc(const float* scores, const int32_t* idx, const
                                   float* loss_per_query, dsa_stream_t stream) {
   if (!scores || !idx || !p_sel || !loss) return DSA_ERR_INVALID_ARG;
   if (B <= 0 || Lq <= 0 || Lk <= 0 || Lq > Lk || k <= 0) return DSA_ERR_INVALID_ARG;
-  if (!aligned16(scores) || !aligned16(idx) || !aligned16(p_sel) || (reinterpret_cast<uintptr_t>(loss) & 3u))
+  if (!aligned16(scores) || !aligned16(idx) || !aligned16(p_sel) || (reinterpret_cast<uintptr_t>(loss) & 3u) ||
+      (loss_per_query && !aligned16(loss_per_query)))
     return DSA_ERR_INVALID_ARG;
   const long rows = static_cast<long>(B) * Lq;
   if (rows > kKlNoAllocMaxRows) return DSA_ERR_UNSUPPORTED;
@@ -500,6 +529,20 @@ dsa_status dsa_indexer_kl_noalloc(const float* scores, const int32_t* idx, const
   if (sr != DSA_OK) return sr;
   return launch(dsa::kl::kl_sum_kernel, 1u, dsa::kl::kSumThreads, 0, st, 1, static_cast<const float*>(per_row),
                 static_cast<int>(rows), loss);
+}
+
+dsa_status dsa_set_wait_limit_ns(uint64_t ns) {
+  const unsigned long long v = ns == 0 ? dsa::kWaitLimitNs : static_cast<unsigned long long>(ns);
+  if (cudaMemcpyToSymbol(dsa::g_wait_limit_ns, &v, sizeof(v)) != cudaSuccess) return DSA_ERR_CUDA;
+  return DSA_OK;
+}
+
+dsa_status dsa_selftest_wait(dsa_stream_t stream) {
+  DeviceInfo dev;
+  const dsa_status ds = current_device(dev);
+  if (ds != DSA_OK) return ds;
+  wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>();
+  return launch_result();
 }
 
 dsa_status dsa_last_device_status(dsa_stream_t stream) {

@@ -105,7 +105,7 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Bounded wait for the phase with the given parity.  Returns false (after recording
-// DSA_ERR_TIMEOUT with `site`) if the phase does not complete within kWaitLimitNs, or if
+// DSA_ERR_TIMEOUT with `site`) if the phase does not complete within wait_limit_ns(), or if
 // another thread of the CTA already gave up (*abort != 0).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           int site) {
@@ -114,7 +114,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
-    if (global_timer_ns() - t0 > kWaitLimitNs) {
+    if (global_timer_ns() - t0 > wait_limit_ns()) {
       record_timeout(site);
       *abort = 1;
       return false;
@@ -219,7 +219,7 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
   while (true) {
     if (mbar_try_wait_cluster(bar, parity)) return true;
     if (*abort) return false;
-    if (global_timer_ns() - t0 > kWaitLimitNs) {
+    if (global_timer_ns() - t0 > wait_limit_ns()) {
       record_timeout(site);
       *abort = 1;
       return false;
@@ -261,7 +261,7 @@ __device__ __forceinline__ void tma_gather4(void* smem_dst, const CUtensorMap* m
 __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
   const uint64_t t0 = global_timer_ns();
   while (!mbar_try_wait(bar, parity)) {
-    if (global_timer_ns() - t0 > kWaitLimitNs) return;
+    if (global_timer_ns() - t0 > wait_limit_ns()) return;
   }
 }
 

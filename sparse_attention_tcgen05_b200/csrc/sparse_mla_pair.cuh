@@ -271,7 +271,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t now = global_timer_ns();
           if (t_idle == 0) {
             t_idle = now;
-          } else if (now - t_idle > kWaitLimitNs) {
+          } else if (now - t_idle > wait_limit_ns()) {
             record_timeout(61);
             *abort_flag = 1;
             goto done;

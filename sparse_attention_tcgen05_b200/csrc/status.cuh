@@ -7,9 +7,15 @@
 
 namespace dsa {
 
-// Upper bound on any single wait inside a kernel (mbarrier phases).  Kernels here finish in
-// milliseconds; a wait this long means a lost arrival, so the kernel records it and exits.
+// Default upper bound on any single wait inside a kernel (mbarrier phases).  Kernels here finish
+// in milliseconds; a wait this long means a lost arrival, so the kernel records it and exits.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+// The bound in force on this device (dsa_set_wait_limit_ns changes it, e.g. so that a test can
+// make a wait expire quickly).  Read only on the slow path of a wait.
+__device__ unsigned long long g_wait_limit_ns = kWaitLimitNs;
+
+__device__ __forceinline__ uint64_t wait_limit_ns() { return g_wait_limit_ns; }
 
 // Low byte: dsa_status code; bits 8..15: the wait site that expired (for diagnostics).
 __device__ int g_device_status;

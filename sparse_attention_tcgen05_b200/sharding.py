@@ -25,9 +25,17 @@ def shard_rows(n_rows: int, rank: int, world: int) -> tuple[int, int]:
     return start, start + base + (1 if rank < extra else 0)
 
 
+# Work of one selected latent entry in the attention relative to one indexer key: 128 heads x
+# (576 + 512) = 139264 bf16 MACs against 64 x 128 = 8192 FP8 MACs, which run at twice the bf16
+# rate ("DeepSeek-V3.2" analysis page, sec. 1.1: the indexer costs about 1/34 of the attention
+# per (t, s) pair).
+MLA_WEIGHT = 128 * (576 + 512) / (64 * 128 / 2)
+
+
 def causal_row_cost(Lq: int, Lk: int, k: int, mla_weight: float = 1.0) -> np.ndarray:
     """Relative work of each query row i of a causal sequence (position t = i + Lk - Lq): the
-    indexer scores t + 1 keys and the attention reads min(k, t + 1) latents."""
+    indexer scores t + 1 keys and the attention reads min(k, t + 1) latents, each weighted by
+    mla_weight (MLA_WEIGHT for the full DSA dimensions)."""
     t = np.arange(Lq, dtype=np.float64) + (Lk - Lq)
     return (t + 1.0) + mla_weight * np.minimum(float(k), t + 1.0)
 
@@ -36,7 +44,13 @@ def shard_causal_rows(Lq: int, Lk: int, k: int, rank: int, world: int,
                       mla_weight: float = 1.0) -> tuple[int, int]:
     """Contiguous query rows [start, stop) of one causal sequence for rank `rank`, cut where the
     running work crosses rank/world of the total, so that late (long) rows are not all on the
-    last rank."""
+    last rank.
+
+    How a rank calls the C ABI for its shard: the ABI places query i at t = i + Lk - Lq, so the
+    rank passes Lq' = stop - start and Lk' = stop + (Lk - Lq), with q_I, w and q sliced to the
+    query rows [start, stop) and k_I and kv truncated to the keys [0, Lk').  Query i of the shard
+    then sits at t = start + i + (Lk - Lq), as in the whole sequence.  Passing the full Lk
+    instead would shift every position."""
     if not 0 <= rank < world:
         raise ValueError(f"rank {rank} outside a world of {world}")
     cum = np.concatenate([[0.0], np.cumsum(causal_row_cost(Lq, Lk, k, mla_weight))])

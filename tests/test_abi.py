@@ -49,6 +49,11 @@ def test_host_validation_rejects_without_touching_a_device(lib):
                                   None, None, None, 0, None) == 1
     assert lib.dsa_indexer_kl(fake, fake, None, 1, 1, 8, 4, fake, None, None, 0, None) == 1
     assert lib.dsa_indexer_kl_noalloc(fake, fake, fake, 1, 4, 2, 4, fake, None, None) == 1
+    # a misaligned per-row output or workspace is refused before any launch
+    odd = P(0x10004)
+    assert lib.dsa_indexer_kl(fake, fake, fake, 1, 4, 8, 4, fake, odd, None, 0, None) == 1
+    assert lib.dsa_indexer_kl(fake, fake, fake, 1, 4, 8, 4, fake, None, odd, 64, None) == 1
+    assert lib.dsa_indexer_kl_noalloc(fake, fake, fake, 1, 4, 8, 4, fake, odd, None) == 1
 
 
 def test_workspace_sizes(lib):
@@ -67,6 +72,8 @@ def test_traffic_hash_ignores_comments_but_not_code():
     spec = importlib.util.spec_from_file_location(
         "bench", os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "bench.py"))
     bench = importlib.util.module_from_spec(spec)
+    import sys
+    bench = sys.modules.setdefault("bench", bench)  # dataclasses look their module up by name
     spec.loader.exec_module(bench)
     src = "int a = 1; // one\n/* block\n comment */ int b = a + 2;\n"
     same = "int a = 1;\n\n   int b = a + 2; // other words\n"

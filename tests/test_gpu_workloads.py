@@ -14,7 +14,7 @@ from tests import parity
 
 pytestmark = pytest.mark.gpu
 
-N_RANDOM_ROWS = int(os.environ.get("DSA_TEST_RANDOM_ROWS", "24"))
+N_RANDOM_ROWS = int(os.environ.get("DSA_TEST_RANDOM_ROWS", "512"))
 
 
 @pytest.fixture(scope="module")
