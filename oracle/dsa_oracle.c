@@ -16,6 +16,9 @@
  *     and L1-normalised, "DSA Continued Pre-Training" page, Stage 1
  *   - sparse-stage indexer loss L^I = sum_t KL(p[t,S_t] || Softmax(I[t,S_t])),
  *     "DSA Continued Pre-Training" page, Stage 2, and the analysis page eq. (4)
+ *   - dense warm-up loss L^I = sum_t KL(p[t,:] || Softmax(I[t,:])) over every s <= t, with p
+ *     the dense main attention summed over heads and L1-normalised, "DSA Continued
+ *     Pre-Training" page, Stage 1, and the analysis page eq. (3)
  *
  * Readings where the pages are silent (each also listed in the design notes):
  *   - causal visibility includes the query's own position: s <= t;
@@ -189,6 +192,53 @@ double ref_kl_row(const double* scores_row, const int32_t* idx, const double* p,
     if (idx[i] < 0 || p[i] == 0.0) continue;
     double log_q = scores_row[idx[i]] - log_z;
     kl += p[i] * (log(p[i]) - log_q);
+  }
+  return kl;
+}
+
+/* ---- f3: dense warm-up target and loss, eq. (3) ------------------------------------------- */
+/* Target of the dense warm-up ("DSA Continued Pre-Training", Stage 1): for query t, the dense
+ * main attention over every s <= t (MQA mode: logits scale * <q[h,:], c[s,:]> over all d_qk
+ * latent dims, softmax over s per head), summed over the H heads and L1-normalised along s.
+ * q_row: [H][d_qk] bf16; kv_seq: [>= t+1][d_qk] bf16; p: [t+1]. */
+void ref_dense_p_row(const uint16_t* q_row, const uint16_t* kv_seq, int t, int H, int d_qk,
+                     double scale, double* p) {
+  int n = t + 1;
+  double* z = (double*)malloc(sizeof(double) * (size_t)n);
+  for (int s = 0; s < n; ++s) p[s] = 0.0;
+  for (int h = 0; h < H; ++h) {
+    double m = -INFINITY;
+    for (int s = 0; s < n; ++s) {
+      double dot = 0.0;
+      for (int d = 0; d < d_qk; ++d)
+        dot += ref_bf16_to_double(q_row[h * d_qk + d]) * ref_bf16_to_double(kv_seq[(int64_t)s * d_qk + d]);
+      z[s] = scale * dot;
+      if (z[s] > m) m = z[s];
+    }
+    double denom = 0.0;
+    for (int s = 0; s < n; ++s) denom += exp(z[s] - m);
+    for (int s = 0; s < n; ++s) p[s] += exp(z[s] - m) / denom;  /* this head's probabilities */
+  }
+  double total = 0.0;
+  for (int s = 0; s < n; ++s) total += p[s];
+  for (int s = 0; s < n; ++s) p[s] /= total;
+  free(z);
+}
+
+/* One row of eq. (3): KL(p[t,:] || Softmax(I[t,:])) over every s <= t, natural log,
+ * 0 * ln 0 = 0.  scores_row: I[t, 0..t]; p: [t+1]. */
+double ref_dense_kl_row(const double* scores_row, int t, const double* p) {
+  int n = t + 1;
+  double m = -INFINITY;
+  for (int s = 0; s < n; ++s)
+    if (scores_row[s] > m) m = scores_row[s];
+  double denom = 0.0;
+  for (int s = 0; s < n; ++s) denom += exp(scores_row[s] - m);
+  double log_z = m + log(denom);
+  double kl = 0.0;
+  for (int s = 0; s < n; ++s) {
+    if (p[s] == 0.0) continue;
+    kl += p[s] * (log(p[s]) - (scores_row[s] - log_z));
   }
   return kl;
 }

@@ -46,6 +46,9 @@ def _load():
         lib.ref_kl_row.argtypes = [vp, vp, vp, i32]
         lib.ref_kl_row.restype = f64
         lib.ref_dense_mla_row.argtypes = [vp, vp, i32, i32, i32, i32, f64, vp, vp, vp]
+        lib.ref_dense_p_row.argtypes = [vp, vp, i32, i32, i32, f64, vp]
+        lib.ref_dense_kl_row.argtypes = [vp, i32, vp]
+        lib.ref_dense_kl_row.restype = f64
         lib.ref_path_rows.argtypes = [vp, vp, vp, vp, vp, i32, vp, i64, i32, i32, i32, i32, i32, i32,
                                       i32, i32, i32, f64, i32, vp, vp, vp, vp, vp, vp, i32]
         _lib = lib
@@ -127,6 +130,24 @@ def dense_mla_row(q_row, kv_seq, t: int, d_v: int, scale: float, want_A: bool = 
     _load().ref_dense_mla_row(qp, kp, t, H, d_qk, d_v, float(scale), out.ctypes.data, lse.ctypes.data,
                               A.ctypes.data if want_A else None)
     return out, lse, A
+
+
+def dense_p_row(q_row, kv_seq, t: int, scale: float) -> np.ndarray:
+    """Dense warm-up target p[t, 0..t]: dense MQA attention over every s <= t, summed over
+    heads, L1-normalised (Stage 1 of "DSA Continued Pre-Training")."""
+    q_row, qp = _c(q_row, np.uint16)
+    kv_seq, kp = _c(kv_seq, np.uint16)
+    H, d_qk = q_row.shape
+    p = np.empty(t + 1, dtype=np.float64)
+    _load().ref_dense_p_row(qp, kp, t, H, d_qk, float(scale), p.ctypes.data)
+    return p
+
+
+def dense_kl_row(scores_row, t: int, p) -> float:
+    """One row of eq. (3): KL(p[t,:] || Softmax(I[t, 0..t]))."""
+    scores_row, sp = _c(scores_row, np.float64)
+    p, pp = _c(p, np.float64)
+    return _load().ref_dense_kl_row(sp, t, pp)
 
 
 def path_rows(wl, rows, qI, kI, w, q, kv, rows_packed: bool, nthreads: int = 1,
