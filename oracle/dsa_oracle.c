@@ -19,6 +19,9 @@
  *   - dense warm-up loss L^I = sum_t KL(p[t,:] || Softmax(I[t,:])) over every s <= t, with p
  *     the dense main attention summed over heads and L1-normalised, "DSA Continued
  *     Pre-Training" page, Stage 1, and the analysis page eq. (3)
+ *   - the gradient of one row's L^I with respect to the indexer's inputs q_I, w and k_I (the
+ *     indexer is trained from L^I alone, on a detached input: "DSA Continued Pre-Training",
+ *     Stage 2), with the selected set held fixed (top-k is piecewise constant)
  *
  * Readings where the pages are silent (each also listed in the design notes):
  *   - causal visibility includes the query's own position: s <= t;
@@ -241,6 +244,99 @@ double ref_dense_kl_row(const double* scores_row, int t, const double* p) {
     kl += p[s] * (log(p[s]) - (scores_row[s] - log_z));
   }
   return kl;
+}
+
+/* ---- f2: gradient of the indexer loss with respect to the indexer's inputs -------------- */
+/* Real-valued inputs (fp64) so that the loss can be differentiated numerically as well:
+ * q_row [H_I][d_I], k_seq [Lk][d_I], w_row [H_I]; idx [k] (-1 = empty slot, the set held fixed);
+ * p [k] the target over the slots.  One row's loss of eq. (4) (eq. (3) when idx lists every
+ * s <= t):  L = sum_i p_i (ln p_i - ln q_i),  q = Softmax_i(I_i),
+ * I_i = sum_j w_j ReLU(q_j . k_{idx_i}). */
+double ref_indexer_loss_row_f64(const double* q_row, const double* k_seq, const double* w_row,
+                                const int32_t* idx, const double* p, int k, int H_I, int d_I) {
+  double* I = (double*)malloc(sizeof(double) * (size_t)(k > 0 ? k : 1));
+  double m = -INFINITY;
+  for (int i = 0; i < k; ++i) {
+    if (idx[i] < 0) continue;
+    double score = 0.0;
+    for (int j = 0; j < H_I; ++j) {
+      double dot = 0.0;
+      for (int d = 0; d < d_I; ++d) dot += q_row[j * d_I + d] * k_seq[(int64_t)idx[i] * d_I + d];
+      score += w_row[j] * (dot > 0.0 ? dot : 0.0);
+    }
+    I[i] = score;
+    if (score > m) m = score;
+  }
+  double denom = 0.0;
+  for (int i = 0; i < k; ++i)
+    if (idx[i] >= 0) denom += exp(I[i] - m);
+  double log_z = m + log(denom);
+  double loss = 0.0;
+  for (int i = 0; i < k; ++i) {
+    if (idx[i] < 0 || p[i] == 0.0) continue;
+    loss += p[i] * (log(p[i]) - (I[i] - log_z));
+  }
+  free(I);
+  return loss;
+}
+
+/* Its gradient, by the chain rule through the definitions above:
+ *   dL/dI_i = q_i * (sum_i' p_i') - p_i                        (softmax and KL)
+ *   dL/dw_j = sum_i dL/dI_i * ReLU(a_ji),   a_ji = q_j . k_{idx_i}
+ *   dL/dq_j = sum_i dL/dI_i * w_j * [a_ji > 0] * k_{idx_i}
+ *   dL/dk_s += sum_{i: idx_i = s} dL/dI_i * sum_j w_j [a_ji > 0] q_j
+ * with ReLU'(0) taken as 0.  dq [H_I][d_I] and dw [H_I] are written; dk [Lk][d_I] is
+ * ACCUMULATED (several query rows add into the same keys); g [k] (nullable) gets dL/dI. */
+void ref_indexer_grad_row(const double* q_row, const double* k_seq, const double* w_row,
+                          const int32_t* idx, const double* p, int k, int H_I, int d_I, double* dq,
+                          double* dw, double* dk, double* g) {
+  double* I = (double*)malloc(sizeof(double) * (size_t)(k > 0 ? k : 1));
+  double* a = (double*)malloc(sizeof(double) * (size_t)(k > 0 ? k : 1) * (size_t)H_I);
+  double m = -INFINITY;
+  for (int i = 0; i < k; ++i) {
+    if (idx[i] < 0) continue;
+    double score = 0.0;
+    for (int j = 0; j < H_I; ++j) {
+      double dot = 0.0;
+      for (int d = 0; d < d_I; ++d) dot += q_row[j * d_I + d] * k_seq[(int64_t)idx[i] * d_I + d];
+      a[(int64_t)i * H_I + j] = dot;
+      score += w_row[j] * (dot > 0.0 ? dot : 0.0);
+    }
+    I[i] = score;
+    if (score > m) m = score;
+  }
+  double denom = 0.0, p_total = 0.0;
+  for (int i = 0; i < k; ++i) {
+    if (idx[i] < 0) continue;
+    denom += exp(I[i] - m);
+    p_total += p[i];
+  }
+  for (int j = 0; j < H_I; ++j) {
+    dw[j] = 0.0;
+    for (int d = 0; d < d_I; ++d) dq[j * d_I + d] = 0.0;
+  }
+  for (int i = 0; i < k; ++i) {
+    if (idx[i] < 0) {
+      if (g) g[i] = 0.0;
+      continue;
+    }
+    double gi = exp(I[i] - m) / denom * p_total - p[i];
+    if (g) g[i] = gi;
+    const double* ks = k_seq + (int64_t)idx[i] * d_I;
+    double* dks = dk + (int64_t)idx[i] * d_I;
+    for (int j = 0; j < H_I; ++j) {
+      double aj = a[(int64_t)i * H_I + j];
+      dw[j] += gi * (aj > 0.0 ? aj : 0.0);
+      if (aj > 0.0) {
+        for (int d = 0; d < d_I; ++d) {
+          dq[j * d_I + d] += gi * w_row[j] * ks[d];
+          dks[d] += gi * w_row[j] * q_row[j * d_I + d];
+        }
+      }
+    }
+  }
+  free(a);
+  free(I);
 }
 
 /* ---- dense causal MQA over all s <= t (for the k >= t+1 and eq. (19)/(20) checks) ------- */

@@ -49,6 +49,9 @@ def _load():
         lib.ref_dense_p_row.argtypes = [vp, vp, i32, i32, i32, f64, vp]
         lib.ref_dense_kl_row.argtypes = [vp, i32, vp]
         lib.ref_dense_kl_row.restype = f64
+        lib.ref_indexer_loss_row_f64.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32]
+        lib.ref_indexer_loss_row_f64.restype = f64
+        lib.ref_indexer_grad_row.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, vp, vp, vp, vp]
         lib.ref_path_rows.argtypes = [vp, vp, vp, vp, vp, i32, vp, i64, i32, i32, i32, i32, i32, i32,
                                       i32, i32, i32, f64, i32, vp, vp, vp, vp, vp, vp, i32]
         _lib = lib
@@ -148,6 +151,37 @@ def dense_kl_row(scores_row, t: int, p) -> float:
     scores_row, sp = _c(scores_row, np.float64)
     p, pp = _c(p, np.float64)
     return _load().ref_dense_kl_row(sp, t, pp)
+
+
+def indexer_loss_row_f64(q_row, k_seq, w_row, idx, p) -> float:
+    """One row's indexer loss from real-valued (fp64) indexer inputs, the selection `idx` fixed."""
+    q_row, qp = _c(q_row, np.float64)
+    k_seq, kp = _c(k_seq, np.float64)
+    w_row, wp = _c(w_row, np.float64)
+    idx, ip = _c(idx, np.int32)
+    p, pp = _c(p, np.float64)
+    H_I, d_I = q_row.shape
+    return _load().ref_indexer_loss_row_f64(qp, kp, wp, ip, pp, idx.shape[0], H_I, d_I)
+
+
+def indexer_grad_row(q_row, k_seq, w_row, idx, p, dk=None):
+    """(dq [H_I, d_I], dw [H_I], dk [Lk, d_I], g [k]) of one row's indexer loss; dk accumulates
+    into the array passed (zeros if None)."""
+    q_row, qp = _c(q_row, np.float64)
+    k_seq, kp = _c(k_seq, np.float64)
+    w_row, wp = _c(w_row, np.float64)
+    idx, ip = _c(idx, np.int32)
+    p, pp = _c(p, np.float64)
+    H_I, d_I = q_row.shape
+    dq = np.empty((H_I, d_I))
+    dw = np.empty(H_I)
+    if dk is None:
+        dk = np.zeros_like(k_seq)
+    assert dk.dtype == np.float64 and dk.flags.c_contiguous and dk.shape == k_seq.shape
+    g = np.empty(idx.shape[0])
+    _load().ref_indexer_grad_row(qp, kp, wp, ip, pp, idx.shape[0], H_I, d_I, dq.ctypes.data, dw.ctypes.data,
+                                 dk.ctypes.data, g.ctypes.data)
+    return dq, dw, dk, g
 
 
 def path_rows(wl, rows, qI, kI, w, q, kv, rows_packed: bool, nthreads: int = 1,
