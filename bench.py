@@ -77,6 +77,17 @@ def algorithmic(wl):
     B, Lq, Lk, k = wl.B, wl.Lq, wl.Lk, wl.k
     t = np.arange(Lq) + (Lk - Lq)
     vis = (t + 1).astype(np.float64)            # visible keys per query
+    if wl.dense:
+        # the dense warm-up step: indexer, dense attention (lse pass, p pass, output) with the
+        # target p written for every (t, s), eq. (3) over every visible pair
+        pairs = B * vis.sum()
+        ix = {"bytes": B * Lk * wl.d_I + B * Lq * wl.H_I * (wl.d_I + 4) + B * Lq * Lk * 4,
+              "macs": pairs * wl.H_I * wl.d_I}
+        dm = {"bytes": 2 * B * Lq * wl.H * wl.d_qk + 2 * B * Lk * wl.d_qk + 2 * B * Lq * wl.H * wl.d_v
+              + 4 * B * Lq * wl.H + 4 * B * Lq * Lk,
+              "macs": pairs * wl.H * (2 * wl.d_qk + wl.d_v)}
+        kl = {"bytes": 8 * pairs, "macs": 0.0}
+        return {"indexer": ix, "dense_mla": dm, "indexer_kl": kl}
     sel = np.minimum(k, t + 1).astype(np.float64)  # selected entries per query
     pairs = B * vis.sum()
     nsel = B * sel.sum()
@@ -141,7 +152,7 @@ def tensor_peak(stage, peaks, sustained):
     bf16 = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
     if stage == "indexer":
         return FP8_OVER_BF16 * bf16
-    if stage == "sparse_mla":
+    if stage in ("sparse_mla", "dense_mla"):
         return bf16
     return None
 
@@ -297,12 +308,14 @@ class Step:
         self.d = {k_: v.to(device) for k_, v in (self.h or h).items()}
         del h
         self.scores = torch.empty(B, Lq, Lk, dtype=torch.float32, device=device)
-        self.idx = torch.empty(B, Lq, wl.k, dtype=torch.int32, device=device)
+        self.idx = None if wl.dense else torch.empty(B, Lq, wl.k, dtype=torch.int32, device=device)
         self.out = torch.empty(B, Lq, wl.H, wl.d_v, dtype=torch.bfloat16, device=device)
         self.lse = torch.empty(B, Lq, wl.H, dtype=torch.float32, device=device)
-        self.p = torch.empty(B, Lq, wl.k, dtype=torch.float32, device=device) if wl.emit_p else None
+        pk = Lk if wl.dense else wl.k  # the dense target covers every position
+        self.p = torch.empty(B, Lq, pk, dtype=torch.float32, device=device) if wl.emit_p else None
         self.loss = torch.empty(1, dtype=torch.float32, device=device)
         nws = max(dsa.dsa_workspace_bytes(dsa.DSA_OP_SPARSE_MLA_FWD, B, Lq, Lk, wl.k, wl.H),
+                  dsa.dsa_workspace_bytes(dsa.DSA_OP_DENSE_MLA_FWD, B, Lq, Lk, 0, wl.H) if wl.dense else 0,
                   dsa.dsa_workspace_bytes(dsa.DSA_OP_INDEXER_KL, B, Lq, Lk, wl.k, 0), 16)
         self.ws = torch.empty(nws, dtype=torch.uint8, device=device)
         if keep_host:
@@ -312,11 +325,12 @@ class Step:
             torch.distributed.get_world_size() > 1
         # the split-KV combine is a separate launch only with more than two splits (two splits
         # combine inside the attention kernel)
-        self.launches_per_step = 3 + (2 if wl.emit_p else 0) + (1 if self._mla_splits() > 2 else 0)
+        self.launches_per_step = (2 if wl.dense else 3) + (2 if wl.emit_p else 0) + \
+            (1 if self._mla_splits() > 2 else 0)
 
     def _mla_splits(self):
         wl = self.wl
-        if wl.emit_p:
+        if wl.emit_p or wl.dense:
             return 1
         ws = self.dsa.dsa_workspace_bytes(self.dsa.DSA_OP_SPARSE_MLA_FWD, wl.B, wl.Lq, wl.Lk, wl.k, wl.H)
         per_split = wl.rows * wl.H * (wl.d_v + 1) * 4  # partial O + lse of one split
@@ -329,6 +343,18 @@ class Step:
         dsa.dsa_indexer(d["qI"], d["kI"], d["w"], self.scores)
         if ev:
             ev[1].record()
+        if wl.dense:  # the dense warm-up step: no selection
+            if ev:
+                ev[2].record()
+            dsa.dsa_dense_mla_fwd(d["q"], d["kv"], wl.scale, self.out, self.lse, self.p, self.ws)
+            if ev:
+                ev[3].record()
+            dsa.dsa_indexer_kl_dense(self.scores, self.p, self.loss, None, self.ws)
+            if self.reduce_loss:
+                sum_over_ranks(self.loss)
+            if ev:
+                ev[4].record()
+            return
         dsa.dsa_topk(self.scores, self.idx)
         if ev:
             ev[2].record()
@@ -418,7 +444,8 @@ def measure(shard, device, steps, warmup, world, peaks, e2e=True):
     step_ms = [a.elapsed_time(b) for a, b in evs]
     # Per-stage times (for the stage roofline fractions) from a separate pass of the same steps
     # with an event between every two launches.
-    stage_ms = {"indexer": [], "topk": [], "sparse_mla": [], "indexer_kl": []}
+    attn = "dense_mla" if wl.dense else "sparse_mla"
+    stage_ms = {"indexer": [], "topk": [], attn: [], "indexer_kl": []}
     for i in range(steps):
         flush.fill_(i & 0xFF)
         e = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
@@ -426,8 +453,10 @@ def measure(shard, device, steps, warmup, world, peaks, e2e=True):
         torch.cuda.synchronize()
         stage_ms["indexer"].append(e[0].elapsed_time(e[1]))
         stage_ms["topk"].append(e[1].elapsed_time(e[2]))
-        stage_ms["sparse_mla"].append(e[2].elapsed_time(e[3]))
+        stage_ms[attn].append(e[2].elapsed_time(e[3]))
         stage_ms["indexer_kl"].append(e[3].elapsed_time(e[4]))
+    if wl.dense:
+        del stage_ms["topk"]
     total_ms = max_over_ranks(sum(step_ms), device)  # the slowest rank's time
     ms_per_step = total_ms / steps
     rows_all = shard.job.rows if world > 1 else wl.rows  # query rows of all ranks
@@ -450,9 +479,12 @@ def measure(shard, device, steps, warmup, world, peaks, e2e=True):
         rec_e2e = {"value": rows_all / (e2e_ms / 1e3), "unit": "query-tokens/s",
                    "h2d_bytes_per_step": step.h2d_bytes(), "d2h_bytes_per_step": step.d2h_bytes()}
 
-    # prefill steps last tens of milliseconds and repeat back to back: their contractions are
-    # held to the sustained (power-capped) GEMM peak; decode steps last microseconds (burst)
-    sustained = wl.Lq > 1 and ms_per_step >= 5.0
+    # contractions are held to the burst GEMM peak (the stricter denominator); the sustained,
+    # power-capped one is used only when the clocks sampled during the steps show the power cap
+    # holding the SM clock well below its maximum
+    c = clk.summary()
+    sustained = bool(c.get("sm_mhz") and c.get("sm_max_mhz") and "sw_power_cap" in c.get("reasons", [])
+                     and c["sm_mhz"] < 0.9 * c["sm_max_mhz"])
     work = algorithmic(wl)
     stages = {}
     for name, ms in stage_ms.items():
@@ -486,7 +518,7 @@ def measure(shard, device, steps, warmup, world, peaks, e2e=True):
             "ms_per_step": ms_per_step, "value": qtok, "unit": "query-tokens/s",
             "path_roofline_us": round(path_roof, 2),
             "path_roofline_frac": round(path_roof / (ms_per_step * 1e3), 4),
-            "stages": stages, "roofline": roof, "clocks": clk.summary(), "e2e": rec_e2e,
+            "stages": stages, "roofline": roof, "clocks": c, "e2e": rec_e2e,
             "gpu_launches": step.launches_per_step * steps}
 
 
@@ -528,8 +560,8 @@ def gpu_arm(args, rank, world, device):
     if world == 1 and not args.no_extra:
         # every other workload, timed the same way (fewer steps, no host round trip)
         extra = {}
-        names = [NORTH_STAR] + [n for n in ("decode_32k", "prefill_2x8k", "indexer_kl_16k", "tiny_prefill")
-                                if n != args.workload]
+        names = [NORTH_STAR] + [n for n in ("decode_32k", "prefill_2x8k", "indexer_kl_16k", "dense_warmup_16k",
+                                            "tiny_prefill") if n != args.workload]
         for name in names:
             if name == args.workload:
                 continue

@@ -17,6 +17,8 @@ sections of the V3.2 analysis page):
   prefill_2x8k      B=2, L=8192 causal, dims of decode_32k
   long_prefill_32k  B=1, L=32768 causal, dims of decode_32k
   indexer_kl_16k    B=1, L=16384 causal, dims of decode_32k, plus p and L^I
+  dense_warmup_16k  B=1, L=16384 causal, dims of decode_32k: the dense warm-up step
+                    (indexer, dense attention with its target p over every s <= t, eq. (3))
 q_I and k_I are integers uniform in [-3, 3] stored as e4m3; q and kv are
 N(0,1) rounded to bf16.  The stream recipe is in gen.c.
 """
@@ -125,6 +127,7 @@ class Workload:
     d_v: int
     scale: float
     emit_p: bool = False
+    dense: bool = False  # the dense warm-up step: no top-k, attention and KL over every s <= t
     notes: str = field(default="", compare=False)
 
     @property
@@ -149,6 +152,8 @@ WORKLOADS = {
                                576, 512, 1.0 / math.sqrt(192.0), emit_p=True),
     "decode_128k": Workload("decode_128k", 0xD5A0 + 6, 32, 1, 131072, 64, 128, 16, 2048, 128, 576, 512,
                             1.0 / math.sqrt(192.0)),
+    "dense_warmup_16k": Workload("dense_warmup_16k", 0xD5A0 + 9, 1, 16384, 16384, 64, 128, 16, 16384, 128,
+                                 576, 512, 1.0 / math.sqrt(192.0), emit_p=True, dense=True),
     # a 4K-token prefill with the full dims: small enough for counter captures (about 1 GB on
     # the device) while its inputs still exceed the 126 MB L2
     "prefill_1x4k": Workload("prefill_1x4k", 0xD5A0 + 8, 1, 4096, 4096, 64, 128, 16, 2048, 128, 576,
@@ -157,10 +162,12 @@ WORKLOADS = {
 
 
 def custom(name: str, seed: int, B: int, Lq: int, Lk: int, H_I: int, d_I: int, w_den: int, k: int,
-           H: int, d_qk: int, d_v: int, scale: float | None = None, emit_p: bool = False) -> Workload:
+           H: int, d_qk: int, d_v: int, scale: float | None = None, emit_p: bool = False,
+           dense: bool = False) -> Workload:
     if scale is None:
         scale = 1.0 / math.sqrt(d_qk)
-    return Workload(name, seed, B, Lq, Lk, H_I, d_I, w_den, k, H, d_qk, d_v, scale, emit_p)
+    return Workload(name, seed, B, Lq, Lk, H_I, d_I, w_den, Lk if dense else k, H, d_qk, d_v, scale,
+                    emit_p or dense, dense)
 
 
 # ---- per-tensor draws ------------------------------------------------------------------------

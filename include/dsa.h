@@ -52,7 +52,14 @@ typedef enum {
 /* A cudaStream_t passed through the ABI without CUDA headers. */
 typedef void* dsa_stream_t;
 
-enum { DSA_OP_INDEXER = 0, DSA_OP_TOPK = 1, DSA_OP_SPARSE_MLA_FWD = 2, DSA_OP_INDEXER_KL = 3 };
+enum {
+  DSA_OP_INDEXER = 0,
+  DSA_OP_TOPK = 1,
+  DSA_OP_SPARSE_MLA_FWD = 2,
+  DSA_OP_INDEXER_KL = 3,
+  DSA_OP_DENSE_MLA_FWD = 4,
+  DSA_OP_INDEXER_KL_DENSE = 5
+};
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char* dsa_status_str(dsa_status s);
@@ -135,6 +142,37 @@ dsa_status dsa_sparse_mla_fwd(const void* q_bf16, const void* kv_bf16, const int
 dsa_status dsa_indexer_kl(const float* scores, const int32_t* idx, const float* p_sel, int B,
                           int Lq, int Lk, int k, float* loss, float* loss_per_query, void* ws,
                           size_t ws_bytes, dsa_stream_t stream);
+
+/*
+ * Dense warm-up, main attention and its target ("DSA Continued Pre-Training" page, Stage 1;
+ * "DeepSeek-V3.2" analysis page, sec. 1.1, the dense warm-up paragraph and eq. (3)): causal MQA
+ * over EVERY position s <= t(i), the attention the indexer is aligned with before top-k
+ * selection is switched on.  Same arithmetic as dsa_sparse_mla_fwd with slot j read as position
+ * j (k = Lk):
+ *   out[b,i,h,:] = sum_{s<=t} P_h,s kv[b,s,0:d_v],  lse[b,i,h] = ln sum_{s<=t} exp(z_h,s)
+ *   p_full[b,i,s] = sum_h P_h,s / H  for s <= t, 0 for s > t   (the target p[t,:] of eq. (3))
+ *   q_bf16 [B,Lq,H,d_qk] bf16, kv_bf16 [B,Lk,d_qk] bf16, out_bf16 [B,Lq,H,d_v] bf16,
+ *   lse [B,Lq,H] fp32 (nullable), p_full [B,Lq,Lk] fp32 (nullable)
+ * Supported: H <= 128, (d_qk, d_v) in {(576, 512), (80, 64)}, Lk <= 65536.
+ * ws: dsa_workspace_bytes(DSA_OP_DENSE_MLA_FWD, B, Lq, Lk, 0, H) bytes.
+ */
+dsa_status dsa_dense_mla_fwd(const void* q_bf16, const void* kv_bf16, int B, int Lq, int Lk, int H,
+                             int d_qk, int d_v, float scale, void* out_bf16, float* lse, float* p_full,
+                             void* ws, size_t ws_bytes, dsa_stream_t stream);
+
+/*
+ * Dense warm-up indexer loss, eq. (3) ("DSA Continued Pre-Training" page, Stage 1):
+ *   L^I = sum_{b,i} sum_{s<=t} p[b,i,s] (ln p[b,i,s] - ln q[b,i,s]),
+ *   q[b,i,:] = Softmax(scores[b,i,0..t]),  0 * ln 0 = 0.
+ *   scores [B,Lq,Lk] fp32 (dsa_indexer's output), p_full [B,Lq,Lk] fp32 (dsa_dense_mla_fwd's),
+ *   loss: one fp32 (device), loss_per_query [B,Lq] fp32 (nullable)
+ * fp32 per-row arithmetic, fixed-order fp64 sum over rows.
+ * ws: dsa_workspace_bytes(DSA_OP_INDEXER_KL_DENSE, B, Lq, Lk, 0, 0) bytes (unused when
+ * loss_per_query is given).
+ */
+dsa_status dsa_indexer_kl_dense(const float* scores, const float* p_full, int B, int Lq, int Lk,
+                                float* loss, float* loss_per_query, void* ws, size_t ws_bytes,
+                                dsa_stream_t stream);
 
 /*
  * The indexer loss of dsa_indexer_kl for callers that cannot hand the library any scratch

@@ -18,14 +18,18 @@ from . import build as _build
 __all__ = [
     "DsaError", "load", "dsa_status_str", "dsa_version", "dsa_workspace_bytes", "dsa_indexer",
     "dsa_topk", "dsa_sparse_mla_fwd", "dsa_indexer_kl", "dsa_indexer_kl_noalloc",
-    "dsa_last_device_status", "dsa_set_wait_limit_ns", "dsa_selftest_wait",
-    "DSA_OP_INDEXER", "DSA_OP_TOPK", "DSA_OP_SPARSE_MLA_FWD", "DSA_OP_INDEXER_KL", "EXPORTED",
+    "dsa_last_device_status", "dsa_set_wait_limit_ns", "dsa_selftest_wait", "dsa_dense_mla_fwd",
+    "dsa_indexer_kl_dense",
+    "DSA_OP_INDEXER", "DSA_OP_TOPK", "DSA_OP_SPARSE_MLA_FWD", "DSA_OP_INDEXER_KL",
+    "DSA_OP_DENSE_MLA_FWD", "DSA_OP_INDEXER_KL_DENSE", "EXPORTED",
 ]
 
 DSA_OP_INDEXER, DSA_OP_TOPK, DSA_OP_SPARSE_MLA_FWD, DSA_OP_INDEXER_KL = 0, 1, 2, 3
+DSA_OP_DENSE_MLA_FWD, DSA_OP_INDEXER_KL_DENSE = 4, 5
 EXPORTED = ("dsa_status_str", "dsa_version", "dsa_workspace_bytes", "dsa_indexer", "dsa_topk",
             "dsa_sparse_mla_fwd", "dsa_indexer_kl", "dsa_indexer_kl_noalloc",
-            "dsa_last_device_status", "dsa_set_wait_limit_ns", "dsa_selftest_wait")
+            "dsa_last_device_status", "dsa_set_wait_limit_ns", "dsa_selftest_wait",
+            "dsa_dense_mla_fwd", "dsa_indexer_kl_dense")
 
 
 class DsaError(RuntimeError):
@@ -60,9 +64,11 @@ def load(rebuild: bool = False) -> ctypes.CDLL:
         lib.dsa_last_device_status.argtypes = [vp]
         lib.dsa_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
         lib.dsa_selftest_wait.argtypes = [vp]
+        lib.dsa_dense_mla_fwd.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, f32, vp, vp, vp, vp, sz, vp]
+        lib.dsa_indexer_kl_dense.argtypes = [vp, vp, i32, i32, i32, vp, vp, vp, sz, vp]
         for name in ("dsa_indexer", "dsa_topk", "dsa_sparse_mla_fwd", "dsa_indexer_kl",
                      "dsa_indexer_kl_noalloc", "dsa_last_device_status", "dsa_set_wait_limit_ns",
-                     "dsa_selftest_wait"):
+                     "dsa_selftest_wait", "dsa_dense_mla_fwd", "dsa_indexer_kl_dense"):
             getattr(lib, name).restype = i32
         _lib = lib
     return _lib
@@ -181,6 +187,44 @@ def dsa_indexer_kl(scores: torch.Tensor, idx: torch.Tensor, p_sel: torch.Tensor,
     _raise("dsa_indexer_kl",
            load().dsa_indexer_kl(_ptr(scores), _ptr(idx), _ptr(p_sel), B, Lq, Lk, k, _ptr(loss),
                                  _ptr(loss_per_query), wsp, wsb, _stream(stream)))
+
+
+def dsa_dense_mla_fwd(q: torch.Tensor, kv: torch.Tensor, scale: float, out: torch.Tensor,
+                      lse: torch.Tensor | None = None, p_full: torch.Tensor | None = None,
+                      ws: torch.Tensor | None = None, stream=None) -> None:
+    """Dense causal MQA of q [B,Lq,H,d_qk] over every kv[b, s<=t] (the dense warm-up's main
+    attention); out [B,Lq,H,d_v] bf16, optional lse [B,Lq,H] and the head-summed target
+    p_full [B,Lq,Lk] (fp32, 0 for s > t)."""
+    B, Lq, H, d_qk = q.shape
+    Lk = kv.shape[1]
+    d_v = out.shape[3]
+    _check(q, "q", torch.bfloat16, (B, Lq, H, d_qk))
+    _check(kv, "kv", torch.bfloat16, (B, Lk, d_qk))
+    _check(out, "out", torch.bfloat16, (B, Lq, H, d_v))
+    if lse is not None:
+        _check(lse, "lse", torch.float32, (B, Lq, H))
+    if p_full is not None:
+        _check(p_full, "p_full", torch.float32, (B, Lq, Lk))
+    wsp, wsb = _ws(ws)
+    _raise("dsa_dense_mla_fwd",
+           load().dsa_dense_mla_fwd(_ptr(q), _ptr(kv), B, Lq, Lk, H, d_qk, d_v, float(scale), _ptr(out),
+                                    _ptr(lse), _ptr(p_full), wsp, wsb, _stream(stream)))
+
+
+def dsa_indexer_kl_dense(scores: torch.Tensor, p_full: torch.Tensor, loss: torch.Tensor,
+                         loss_per_query: torch.Tensor | None = None, ws: torch.Tensor | None = None,
+                         stream=None) -> None:
+    """loss[0] = sum over rows of KL(p_full[t, 0..t] || Softmax(scores[t, 0..t])) (eq. (3))."""
+    B, Lq, Lk = scores.shape
+    _check(scores, "scores", torch.float32, (B, Lq, Lk))
+    _check(p_full, "p_full", torch.float32, (B, Lq, Lk))
+    _check(loss, "loss", torch.float32, (1,))
+    if loss_per_query is not None:
+        _check(loss_per_query, "loss_per_query", torch.float32, (B, Lq))
+    wsp, wsb = _ws(ws)
+    _raise("dsa_indexer_kl_dense",
+           load().dsa_indexer_kl_dense(_ptr(scores), _ptr(p_full), B, Lq, Lk, _ptr(loss),
+                                       _ptr(loss_per_query), wsp, wsb, _stream(stream)))
 
 
 def dsa_indexer_kl_noalloc(scores: torch.Tensor, idx: torch.Tensor, p_sel: torch.Tensor,

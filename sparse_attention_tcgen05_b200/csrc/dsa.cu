@@ -151,6 +151,7 @@ dsa_status launch_indexer(const void* q, const void* kk, const float* w, float* 
                  D_I, dsa::indexer::kTileKeys, swz))
     return DSA_ERR_CUDA;
   dsa::indexer::Params p{};
+  p.k = static_cast<const uint8_t*>(kk);
   p.w = w;
   p.scores = scores;
   p.B = B;
@@ -241,7 +242,7 @@ size_t mla_ws_bytes(int rows, int k, int H, int d_v, int sms) {
 template <int D_QK, int D_V>
 dsa_status launch_mla(const void* q, const void* kv, const int32_t* idx, int B, int Lq, int Lk,
                       int H, int k, float scale, void* out, float* lse, float* p_sel, void* ws,
-                      size_t ws_bytes, int sms, cudaStream_t stream) {
+                      size_t ws_bytes, int sms, cudaStream_t stream, int dense = 0) {
   using Cfg = dsa::mla::Cfg<D_QK, D_V>;
   const int rows = B * Lq;
   const MlaSplit sp = mla_split(rows, k, Cfg::kNdv, sms, p_sel != nullptr);
@@ -260,6 +261,7 @@ dsa_status launch_mla(const void* q, const void* kv, const int32_t* idx, int B, 
   p.n_split = sp.n_split;
   p.per_split = sp.per_split;
   p.scale_log2 = scale * dsa::mla::kLog2e;
+  p.dense = dense;
   if (sp.n_split > 1) {
     const size_t need = static_cast<size_t>(sp.n_split) * rows * H * (static_cast<size_t>(D_V) + 1) * sizeof(float);
     if (ws == nullptr || ws_bytes < need || !aligned16(ws)) return DSA_ERR_INVALID_ARG;
@@ -382,7 +384,6 @@ const char* dsa_status_str(dsa_status s) {
 int dsa_version(void) { return 101; }
 
 size_t dsa_workspace_bytes(int op, int B, int Lq, int Lk, int k, int H) {
-  (void)Lk;
   if (B <= 0 || Lq <= 0) return 0;
   const long rows = static_cast<long>(B) * Lq;
   switch (op) {
@@ -393,7 +394,14 @@ size_t dsa_workspace_bytes(int op, int B, int Lq, int Lk, int k, int H) {
       return std::max(mla_ws_bytes(static_cast<int>(rows), k, H, 512, sms),
                       mla_ws_bytes(static_cast<int>(rows), k, H, 64, sms));
     }
+    case DSA_OP_DENSE_MLA_FWD: {
+      if (Lk <= 0 || H <= 0) return 0;
+      const int sms = sm_count_or_default();
+      return std::max(mla_ws_bytes(static_cast<int>(rows), Lk, H, 512, sms),
+                      mla_ws_bytes(static_cast<int>(rows), Lk, H, 64, sms));
+    }
     case DSA_OP_INDEXER_KL:
+    case DSA_OP_INDEXER_KL_DENSE:
       return static_cast<size_t>(rows) * sizeof(float);
     default:
       return 0;
@@ -498,7 +506,7 @@ dsa_status dsa_indexer_kl(const float* scores, const int32_t* idx, const float* 
   if (ds != DSA_OK) return ds;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const dsa_status sr = launch(dsa::kl::kl_rows_kernel, static_cast<unsigned>(rows), dsa::kl::kRowThreads, 0, st, 1,
-                               scores, idx, p_sel, Lk, k, per_row);
+                               scores, idx, p_sel, Lq, Lk, k, per_row);
   if (sr != DSA_OK) return sr;
   return launch(dsa::kl::kl_sum_kernel, 1u, dsa::kl::kSumThreads, 0, st, 1, static_cast<const float*>(per_row),
                 static_cast<int>(rows), loss);
@@ -525,7 +533,58 @@ dsa_status dsa_indexer_kl_noalloc(const float* scores, const int32_t* idx, const
   // Every row's term is written before the sum reads it, so the shared array needs no clearing.
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const dsa_status sr = launch(dsa::kl::kl_rows_kernel, static_cast<unsigned>(rows), dsa::kl::kRowThreads, 0, st, 1,
-                               scores, idx, p_sel, Lk, k, per_row);
+                               scores, idx, p_sel, Lq, Lk, k, per_row);
+  if (sr != DSA_OK) return sr;
+  return launch(dsa::kl::kl_sum_kernel, 1u, dsa::kl::kSumThreads, 0, st, 1, static_cast<const float*>(per_row),
+                static_cast<int>(rows), loss);
+}
+
+dsa_status dsa_dense_mla_fwd(const void* q_bf16, const void* kv_bf16, int B, int Lq, int Lk, int H,
+                             int d_qk, int d_v, float scale, void* out_bf16, float* lse, float* p_full,
+                             void* ws, size_t ws_bytes, dsa_stream_t stream) {
+  if (!q_bf16 || !kv_bf16 || !out_bf16) return DSA_ERR_INVALID_ARG;
+  if (B <= 0 || Lq <= 0 || Lk <= 0 || Lq > Lk || H <= 0) return DSA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q_bf16) || !aligned16(kv_bf16) || !aligned16(out_bf16) || (lse && !aligned16(lse)) ||
+      (p_full && !aligned16(p_full)))
+    return DSA_ERR_INVALID_ARG;
+  if (H > 128 || Lk > 65536 || static_cast<long>(B) * Lk >= INT32_MAX) return DSA_ERR_UNSUPPORTED;
+  if (static_cast<long>(B) * Lq * H * 2 * 8 > INT32_MAX) return DSA_ERR_UNSUPPORTED;
+  DeviceInfo dev;
+  const dsa_status ds = current_device(dev);
+  if (ds != DSA_OK) return ds;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // dense causal attention = the selection kernel with slot j read as position j (k = Lk)
+  if (d_qk == 576 && d_v == 512)
+    return launch_mla<576, 512>(q_bf16, kv_bf16, nullptr, B, Lq, Lk, H, Lk, scale, out_bf16, lse, p_full, ws,
+                                ws_bytes, dev.sms, st, 1);
+  if (d_qk == 80 && d_v == 64)
+    return launch_mla<80, 64>(q_bf16, kv_bf16, nullptr, B, Lq, Lk, H, Lk, scale, out_bf16, lse, p_full, ws,
+                              ws_bytes, dev.sms, st, 1);
+  return DSA_ERR_UNSUPPORTED;
+}
+
+dsa_status dsa_indexer_kl_dense(const float* scores, const float* p_full, int B, int Lq, int Lk, float* loss,
+                                float* loss_per_query, void* ws, size_t ws_bytes, dsa_stream_t stream) {
+  if (!scores || !p_full || !loss) return DSA_ERR_INVALID_ARG;
+  if (B <= 0 || Lq <= 0 || Lk <= 0 || Lq > Lk) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(scores) || !aligned16(p_full) || (reinterpret_cast<uintptr_t>(loss) & 3u) ||
+      (loss_per_query && !aligned16(loss_per_query)))
+    return DSA_ERR_INVALID_ARG;
+  const long rows = static_cast<long>(B) * Lq;
+  if (rows > INT32_MAX) return DSA_ERR_UNSUPPORTED;
+  float* per_row = loss_per_query;
+  if (per_row == nullptr) {
+    if (ws == nullptr || ws_bytes < static_cast<size_t>(rows) * sizeof(float) || !aligned16(ws))
+      return DSA_ERR_INVALID_ARG;
+    per_row = static_cast<float*>(ws);
+  }
+  DeviceInfo dev;
+  const dsa_status ds = current_device(dev);
+  if (ds != DSA_OK) return ds;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const dsa_status sr = launch(dsa::kl::kl_rows_kernel, static_cast<unsigned>(rows), dsa::kl::kRowThreads, 0, st, 1,
+                               scores, static_cast<const int32_t*>(nullptr), p_full, Lq, Lk, Lk, per_row);
   if (sr != DSA_OK) return sr;
   return launch(dsa::kl::kl_sum_kernel, 1u, dsa::kl::kSumThreads, 0, st, 1, static_cast<const float*>(per_row),
                 static_cast<int>(rows), loss);

@@ -8,7 +8,11 @@
 //
 // Persistent, warp-specialised CTA (one per SM):
 //   warp 0        TMA producer: the q_I group once per work item, then k_I tiles (12 stages
-//                 for decode, 6 otherwise)
+//                 for decode, 6 otherwise).  For decode (one query per tile, a pure stream of
+//                 k_I) warps 0, 2 and 3 load the k_I tiles with 16-byte cp.async copies written
+//                 straight into the 128B-swizzled layout instead: plain loads stream from HBM
+//                 faster than TMA tile copies on B200 (about 6.0 against 5.5 TB/s for a 512 MiB
+//                 read), and decode is bound by that stream.
 //   warp 1        MMA issuer (one thread): d_I/32 MMAs of 128 x N x 32 per tile
 //   warp 2        TMEM allocator (2 accumulators of N columns, double-buffered)
 //   warps 4..11   epilogue: tcgen05.ld -> ReLU * w -> head sum -> mask -> store
@@ -28,6 +32,7 @@ constexpr int kThreads = 128 + kEpiWarps * 32;
 constexpr int kTileKeys = 128;
 
 struct Params {
+  const uint8_t* k;  // k_I [B * Lk, d_I] (the decode loads read it directly)
   const float* w;
   float* scores;
   int B, Lq, Lk;
@@ -38,11 +43,18 @@ struct Params {
   int n_items;
 };
 
+// Decode k_I producers (cp.async): warps 0, 2 and 3, and how many tiles each keeps in flight
+// before it signals the oldest one.
+constexpr int kLoadThreads = 96;
+constexpr int kLoadLag = 6;
+
 template <int H_I, int D_I, int G>
 struct Cfg {
   // k_I ring depth: decode streams k_I from HBM with little else per tile, so it keeps twice
   // as many tiles in flight
   static constexpr int kStages = (G == 1) ? 12 : 6;
+  static constexpr bool kCpAsyncK = (G == 1) && (D_I == 128);  // decode: k_I by cp.async
+  static_assert(!kCpAsyncK || kLoadLag < kStages, "the producer signals tile j - lag before reusing stage j");
   static constexpr int N = G * H_I;                      // MMA N (columns per accumulator)
   static constexpr int kQBytes = N * D_I;                // q_I group tile
   static constexpr int kKBytes = kTileKeys * D_I;        // k_I tile
@@ -118,7 +130,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
-      mbar_init(&k_full[s], 1);
+      mbar_init(&k_full[s], C::kCpAsyncK ? kLoadThreads : 1);
       mbar_init(&k_empty[s], 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -139,7 +151,72 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
   pdl_wait();  // first global access below
 
-  if (warp == 0) {
+  if (C::kCpAsyncK && (warp == 0 || warp == 2 || warp == 3)) {
+    // ------------------------------------------------------------------ decode producer
+    // Lane 0 of warp 0 loads each item's q_I group by TMA; the 96 threads load the k_I tiles:
+    // thread pt copies the 16-byte chunks pt, pt + 96, ... of a tile (consecutive threads read
+    // consecutive bytes), each to its 128B-swizzled place.  A thread signals tile j on the
+    // tile's barrier once its copies of tile j have landed (cp.async.wait_group) and are made
+    // visible to the tensor cores' async proxy, which it checks after issuing tile j + lag;
+    // tile j + kStages waits for tile j to be consumed, which needs j signalled (lag < stages).
+    const int pt = (warp == 0 ? 0 : warp - 1) * 32 + lane;
+    const size_t k_rows = static_cast<size_t>(p.B) * p.Lk;
+    int ks = 0, sig = 0;  // stage of the next tile; stage of the oldest unsignalled tile
+    uint32_t kph = 0;
+    int pending = 0;      // tiles issued but not signalled by this thread
+    int qi = 0;
+    bool ok = true;
+    if (warp == 0 && lane == 0) tma_prefetch_desc(&tm_q);
+    for (int u = blockIdx.x; ok && u < p.n_items; u += gridDim.x) {
+      int b, qg, kc, kt0, kt1, n_comp;
+      decode_item(p, u, b, qg, kc);
+      item_tiles<G>(p, qg, kc, kt0, kt1, n_comp);
+      if (n_comp == 0) continue;
+      if (warp == 0 && lane == 0) {
+        const int qb = qi & 1;
+        const uint32_t qph = (qi >> 1) & 1;
+        if (!mbar_wait(&q_empty[qb], qph ^ 1, abort_flag, 1)) ok = false;
+        if (ok) {
+          mbar_arrive_expect_tx(&q_full[qb], C::kQBytes);
+          tma_load_2d(sQ + qb * ((C::kQBytes + 1023) / 1024) * 1024, &tm_q, &q_full[qb], 0,
+                      (b * p.Lq + qg * G) * H_I);
+        }
+      }
+      ++qi;
+      for (int tt = 0; ok && tt < n_comp; ++tt) {
+        if (!mbar_wait(&k_empty[ks], kph ^ 1, abort_flag, 2)) {
+          ok = false;
+          break;
+        }
+        const size_t row0 = static_cast<size_t>(b) * p.Lk + static_cast<size_t>(kt0 + tt) * kTileKeys;
+        const uint32_t dst = smem_u32(sK + ks * C::kKBytes);
+        for (int c = pt; c < kTileKeys * (D_I / 16); c += kLoadThreads) {
+          const int r = c >> 3, ch = c & 7;
+          const bool valid = row0 + r < k_rows;  // rows past the tensor are zero-filled
+          cp_async_16(dst + swizzled_offset(r, ch, 128), p.k + (valid ? (row0 + r) * D_I + ch * 16 : 0), valid);
+        }
+        cp_async_commit();
+        if (++pending > kLoadLag) {
+          cp_async_wait_group<kLoadLag>();
+          fence_proxy_async_smem();
+          mbar_arrive(&k_full[sig]);
+          if (++sig == C::kStages) sig = 0;
+          --pending;
+        }
+        if (++ks == C::kStages) {
+          ks = 0;
+          kph ^= 1;
+        }
+      }
+    }
+    // the remaining tiles (also after an abort: nothing of ours may land after exit)
+    cp_async_wait_group<0>();
+    fence_proxy_async_smem();
+    for (; pending > 0; --pending) {
+      mbar_arrive(&k_full[sig]);
+      if (++sig == C::kStages) sig = 0;
+    }
+  } else if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);

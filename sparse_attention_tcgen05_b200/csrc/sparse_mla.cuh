@@ -49,7 +49,25 @@ struct Params {
   float scale_log2;        // softmax scale * log2(e)
   int fuse2;               // 576-d pair kernel, n_split == 2: both splits of a row form one
                            // cluster of four and combine in the kernel (no combine launch)
+  int dense;               // dense causal attention: no idx, slot j is position j for j <= t,
+                           // k == Lk (the dense warm-up's main attention and its target p)
 };
+
+// Query row served by the r-th row of the grid: in dense mode the latest (longest) rows go
+// first, so that the shortest ones fill the tail.
+__device__ __forceinline__ int work_row(const Params& p, int r) { return p.dense ? p.B * p.Lq - 1 - r : r; }
+
+// Latent position of selection slot `slot` of a row: the caller's index, or the slot itself in
+// dense mode.
+__device__ __forceinline__ int slot_position(const Params& p, const int32_t* idx_row, int slot) {
+  return p.dense ? slot : __ldg(idx_row + slot);
+}
+
+// Dense mode: slots [e0, e1) of row `row` that hold visible positions (s <= t).
+__device__ __forceinline__ int dense_len(const Params& p, int row, int e0, int e1) {
+  const int t = (row % p.Lq) + p.Lk - p.Lq;
+  return max(0, min(e1, t + 1) - e0);
+}
 
 template <int D_QK, int D_V>
 struct Cfg {
@@ -121,9 +139,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   // CTA -> (query row, value-dim half, split)
   const int hv = blockIdx.x % C::kNdv;
   const int split = (blockIdx.x / C::kNdv) % p.n_split;
-  const int row = blockIdx.x / (C::kNdv * p.n_split);
+  const int row = work_row(p, blockIdx.x / (C::kNdv * p.n_split));
   const int b = row / p.Lq;
-  const int32_t* idx_row = p.idx + static_cast<size_t>(row) * p.k;
+  const int32_t* idx_row = p.dense ? nullptr : p.idx + static_cast<size_t>(row) * p.k;
   const int e0 = split * p.per_split;
   const int e1 = min(p.k, e0 + p.per_split);
 
@@ -153,7 +171,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem_s = tmem_base + C::kDvCta;
 
   // Effective length: slots after the last valid one in [e0, e1) need no work.
-  {
+  if (!p.dense) {
     int last = -1;
     for (int x = e0 + static_cast<int>(threadIdx.x); x < e1; x += kThreads)
       if (__ldg(idx_row + x) >= 0) last = x;
@@ -162,7 +180,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0 && last >= 0) atomicMax(s_len, last - e0 + 1);
     __syncthreads();
   }
-  const int len = *s_len;
+  const int len = p.dense ? dense_len(p, row, e0, e1) : *s_len;
   const int nblk = (len + kBN - 1) / kBN;
   Steps st;
   st.n_main = nblk;
@@ -233,7 +251,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int r = c / C::kChunksPerRow;
         const int ch = c - r * C::kChunksPerRow;
         const int slot = e0 + blk * kBN + r;
-        const int s = (slot < e0 + len) ? __ldg(idx_row + slot) : -1;
+        const int s = (slot < e0 + len) ? slot_position(p, idx_row, slot) : -1;
         const bool valid = static_cast<unsigned>(s) < static_cast<unsigned>(p.Lk);
         if (s >= p.Lk) record_bad_index();
         const __nv_bfloat16* srcp = kv_seq + static_cast<size_t>(valid ? s : 0) * D_QK + ch * 8;
@@ -261,7 +279,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t ph = (q >> 1) & 1;
       const int blk = st.block(q);
       const int slot = e0 + blk * kBN + lane;
-      const int sidx = (slot < e0 + len) ? __ldg(idx_row + slot) : -1;
+      const int sidx = (slot < e0 + len) ? slot_position(p, idx_row, slot) : -1;
       const bool svalid = static_cast<unsigned>(sidx) < static_cast<unsigned>(p.Lk);
       const uint32_t vmask = __ballot_sync(0xFFFFFFFFu, svalid);
       if (ok && !mbar_wait(&s_full[sb], ph, abort_flag, 25)) ok = false;

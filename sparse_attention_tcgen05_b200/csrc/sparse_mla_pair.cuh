@@ -17,11 +17,12 @@
 // Q, 128 heads x 288 bf16, as the A operand of S = Q K^T [320, 464), and P 2 x 16 [464, 496)
 // (bf16, the A operand of O += P V).  Keeping Q in tensor memory means S only streams the
 // gathered tile (36 KB per pair of blocks) from shared memory, and leaves shared memory to
-// the 3-stage gather ring and the partial-S exchange buffers.
+// the 4-stage gather ring and the partial-S receive slots (which also stage the outgoing
+// partials, see the exchange argument in the softmax role).
 //
 // Pipeline (per CTA, blocks of 32 selected entries; a p sweep revisits every block):
 //   gather warps   TMA tile::gather4: 4 selected rows per instruction, landing in the
-//                  swizzled K-major tiles the MMA reads (3 stages of a pair of blocks, 80
+//                  swizzled K-major tiles the MMA reads (4 stages of a pair of blocks, 80
 //                  instructions each); all seven warps share every stage.
 //   MMA thread     polls: S = Q K^T of a pair of blocks (N = 64) as soon as its stage landed
 //                  and the previous pair's S was read;
@@ -47,7 +48,7 @@ using mla::named_bar_sync;
 
 constexpr int kBN = 32;             // selected entries per softmax block
 constexpr int kPairN = 2 * kBN;     // entries per gathered stage and per S = Q K^T (MMA N = 64)
-constexpr int kStages = 3;          // gather ring depth (pairs of blocks)
+constexpr int kStages = 4;          // gather ring depth (pairs of blocks)
 constexpr int kRecvSlots = 4;       // partial-S receive slots (see the exchange argument below)
 constexpr int kThreads = 512;       // warps 0-7 softmax, 8 MMA, 9-15 gather
 constexpr int kSoftmaxThreads = 256;  // two warpgroups taking turns by block
@@ -61,9 +62,9 @@ constexpr int kRopeTile = kPairN * 64;              // 64 entries x 32 dims (SW6
 constexpr int kKvStage = 4 * kMainBox + kRopeTile;  // 36 KB
 constexpr int kXSlot = 128 * kBN * 4;               // one partial S (fp32, 16 KB)
 constexpr int kOffKV = 0;
-constexpr int kOffX = kOffKV + kStages * kKvStage;  // [kRecvSlots] the peer's partials
-constexpr int kOffXs = kOffX + kRecvSlots * kXSlot; // [2] own partials staged for the bulk copy
-constexpr int kOffRef = kOffXs + 2 * kXSlot;      // [2][128] per-row reference of a block
+constexpr int kOffX = kOffKV + kStages * kKvStage;  // [kRecvSlots] the peer's partials; slot
+                                                    // (q + 2) % 4 also stages block q's own
+constexpr int kOffRef = kOffX + kRecvSlots * kXSlot;  // [2][128] per-row reference of a block
 constexpr int kOffRed = kOffRef;                   // [2 groups][4 warps][32] p partial sums: the p
                                                    // sweep starts after every reference was read
 constexpr int kOffFin = kOffRef + 2 * 128 * 4;     // [2 groups][2][128] final (l, reference)
@@ -129,9 +130,10 @@ __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint3
 }
 
 // The 32 idx slots of block `blk` as seen by lane `lane` (-1 past the effective length).
-__device__ __forceinline__ int block_slot(const int32_t* idx_row, int e0, int len, int blk, int lane) {
+__device__ __forceinline__ int block_slot(const Params& p, const int32_t* idx_row, int e0, int len, int blk,
+                                          int lane) {
   const int slot = e0 + blk * kBN + lane;
-  return (slot < e0 + len) ? __ldg(idx_row + slot) : -1;
+  return (slot < e0 + len) ? mla::slot_position(p, idx_row, slot) : -1;
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -144,7 +146,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sKV = smem + kOffKV;
   float* sX = reinterpret_cast<float*>(smem + kOffX);
-  uint8_t* sXs = smem + kOffXs;
   float* sRed = reinterpret_cast<float*>(smem + kOffRed);
   float* sRef = reinterpret_cast<float*>(smem + kOffRef);
   float* sFin = reinterpret_cast<float*>(smem + kOffFin);
@@ -171,9 +172,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int pair = blockIdx.x >> 1;
   const int split = pair % p.n_split;
-  const int row = pair / p.n_split;
+  const int row = mla::work_row(p, pair / p.n_split);
   const int b = row / p.Lq;
-  const int32_t* idx_row = p.idx + static_cast<size_t>(row) * p.k;
+  const int32_t* idx_row = p.dense ? nullptr : p.idx + static_cast<size_t>(row) * p.k;
   const int e0 = split * p.per_split;
   const int e1 = min(p.k, e0 + p.per_split);
 
@@ -217,7 +218,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   // Effective length: slots after the last valid one in [e0, e1) need no work (same on both).
-  {
+  if (!p.dense) {
     int last = -1;
     for (int x = e0 + static_cast<int>(threadIdx.x); x < e1; x += kThreads)
       if (__ldg(idx_row + x) >= 0) last = x;
@@ -226,7 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0 && last >= 0) atomicMax(s_len, last - e0 + 1);
     __syncthreads();
   }
-  const int len = *s_len;
+  const int len = p.dense ? mla::dense_len(p, row, e0, e1) : *s_len;
   const int nblk = (len + kBN - 1) / kBN;
   const int total = nblk + ((p.p_sel != nullptr) ? nblk : 0);  // the p sweep revisits every block
 
@@ -300,7 +301,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const CUtensorMap* tmap = bx < 4 ? &tm_main : &tm_rope;
     const uint32_t dst_off = bx < 4 ? static_cast<uint32_t>(bx * kMainBox + g * 512) : static_cast<uint32_t>(4 * kMainBox + g * 256);
     const int npairs = (total + 1) / 2;
-    auto slot_of = [&](int j) { return j < total ? block_slot(idx_row, e0, len, j < nblk ? j : j - nblk, lane) : -1; };
+    auto slot_of = [&](int j) { return j < total ? block_slot(p, idx_row, e0, len, j < nblk ? j : j - nblk, lane) : -1; };
     int next_lo = (total > 0) ? slot_of(0) : -1, next_hi = (total > 1) ? slot_of(1) : -1;
     int issued = 0;
     if (lane == 0) {
@@ -361,7 +362,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const size_t orow = static_cast<size_t>(row) * p.H + h;
     const bool head_ok = h < p.H;
     const int bar_xs = kBarXs0 + wg, bar_red = kBarRed0 + wg;
-    uint8_t* stg_row = sXs + wg * kXSlot + h * (kBN * 4);  // this group's staging slot, row h
     bool ok = true;
 
     // This CTA's 288 dims of Q into tensor memory: dims [8j, 8j+8) of the slice -> columns
@@ -403,12 +403,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
 
     // Steps 1-2 for block q: z[] = the full S(q) (unscaled), -inf at invalid slots.
-    // Staging: one slot per group, reused every other block; the group's leader waits until its
-    // previous copy has read the slot, and a barrier publishes that before anyone rewrites it.
     // Receive slots q % 4: four make reuse safe without a back-signal.  This group sends block
     // q+4 only after it received the peer group's block q+2, which that group sends only after
     // it finished reading the slot of block q.
+    // Staging: the own partial of block q goes out from this CTA's receive slot (q + 2) % 4.  This
+    // group finished reading it (the peer's block q-2) before starting block q, and the peer
+    // writes it next with its block q+2, which it sends only after it received this group's
+    // block q - that is, after the bulk copy read the staged rows.  The group's leader also waits
+    // until its previous copy has read its source before the slot is rewritten.
     auto full_s = [&](int q, uint32_t vm, float (&z)[32]) {
+      uint8_t* stg = reinterpret_cast<uint8_t*>(sX) + ((q + 2) % kRecvSlots) * kXSlot;
+      uint8_t* stg_row = stg + h * (kBN * 4);
       if (wtid == 0) bulk_wait_read_all();
       named_bar_sync(bar_xs, 128);
       uint32_t v[32];
@@ -433,7 +438,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int sl = q % kRecvSlots;
       if (wtid == 0) {
         if (ok)
-          bulk_copy_to_peer(peer_recv + static_cast<uint32_t>(sl * kXSlot), smem_u32(sXs + wg * kXSlot), kXSlot,
+          bulk_copy_to_peer(peer_recv + static_cast<uint32_t>(sl * kXSlot), smem_u32(stg), kXSlot,
                             peer_x_full + sl * 8);
         bulk_commit_group();
         mbar_arrive_expect_tx(&x_full[sl], kXSlot);
@@ -552,12 +557,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
 
     // mask of this group's next block and the pending slot load of the one after
-    uint32_t m_cur = mask_of((wg < total) ? block_slot(idx_row, e0, len, blk_of(wg), lane) : -1);
-    int s_pf = (wg + 2 < total) ? block_slot(idx_row, e0, len, blk_of(wg + 2), lane) : -1;
+    uint32_t m_cur = mask_of((wg < total) ? block_slot(p, idx_row, e0, len, blk_of(wg), lane) : -1);
+    int s_pf = (wg + 2 < total) ? block_slot(p, idx_row, e0, len, blk_of(wg + 2), lane) : -1;
     for (int q = wg; q < total; q += 2) {
       const uint32_t vm = m_cur;
       m_cur = mask_of(s_pf);
-      s_pf = (q + 4 < total) ? block_slot(idx_row, e0, len, blk_of(q + 4), lane) : -1;
+      s_pf = (q + 4 < total) ? block_slot(p, idx_row, e0, len, blk_of(q + 4), lane) : -1;
       if (q >= nblk && !fin) {
         finish();
         fin = true;

@@ -54,11 +54,51 @@ class DeviceWorkload:
         return self.kv.view(torch.int16).cpu().numpy().view(np.uint16)
 
 
+def run_dense_path(dw: DeviceWorkload):
+    """The dense warm-up step through the C ABI: indexer -> dense attention with the target
+    p over every s <= t -> eq. (3) loss; returns device tensors."""
+    import sparse_attention_tcgen05_b200 as dsa
+
+    wl = dw.wl
+    dev = dw.qI.device
+    scores = torch.empty(wl.B, wl.Lq, wl.Lk, dtype=torch.float32, device=dev)
+    out = torch.empty(wl.B, wl.Lq, wl.H, wl.d_v, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(wl.B, wl.Lq, wl.H, dtype=torch.float32, device=dev)
+    p_full = torch.empty(wl.B, wl.Lq, wl.Lk, dtype=torch.float32, device=dev)
+    ws_bytes = dsa.dsa_workspace_bytes(dsa.DSA_OP_DENSE_MLA_FWD, wl.B, wl.Lq, wl.Lk, 0, wl.H)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+    loss = torch.empty(1, dtype=torch.float32, device=dev)
+    per = torch.empty(wl.B, wl.Lq, dtype=torch.float32, device=dev)
+    dsa.dsa_indexer(dw.qI, dw.kI, dw.w, scores)
+    dsa.dsa_dense_mla_fwd(dw.q, dw.kv, wl.scale, out, lse, p_full, ws)
+    dsa.dsa_indexer_kl_dense(scores, p_full, loss, per)
+    assert dsa.dsa_last_device_status() == 0
+    return {"scores": scores, "out": out, "lse": lse, "p_full": p_full, "loss": loss, "loss_rows": per}
+
+
+def oracle_dense_row(dw: DeviceWorkload, r: int, kv_np=None):
+    """The oracle's dense warm-up results for flat row r: scores, out, lse, p[0..t], KL."""
+    from oracle import oracle as ref
+
+    wl = dw.wl
+    b, i = divmod(r, wl.Lq)
+    t = wl.t_of(i)
+    kv = dsa_inputs.kv_latent(wl, b) if kv_np is None else kv_np[b]
+    q = dsa_inputs.q_attn(wl, r, 1)[0]
+    sc = ref.indexer_row(dw.qI_np.reshape(wl.rows, wl.H_I, wl.d_I)[r], dw.kI_np[b],
+                         dw.w_np.reshape(wl.rows, wl.H_I)[r], t)
+    out, lse, _ = ref.dense_mla_row(q, kv, t, wl.d_v, wl.scale)
+    p = ref.dense_p_row(q, kv, t, wl.scale)
+    return {"scores": sc, "out": out, "lse": lse, "p": p, "kl": ref.dense_kl_row(sc, t, p), "t": t}
+
+
 def run_path(dw: DeviceWorkload, emit_p: bool | None = None):
     """indexer -> top-k -> sparse MLA [-> KL] through the C ABI; returns device tensors."""
     import sparse_attention_tcgen05_b200 as dsa
 
     wl = dw.wl
+    if wl.dense:
+        return run_dense_path(dw)
     emit_p = wl.emit_p if emit_p is None else emit_p
     dev = dw.qI.device
     scores = torch.empty(wl.B, wl.Lq, wl.Lk, dtype=torch.float32, device=dev)
