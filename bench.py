@@ -103,6 +103,9 @@ def algorithmic(wl):
         ml["macs"] += nsel * wl.H * wl.d_qk
         ml["bytes"] += 4 * B * Lq * k
     kl = {"bytes": 4 * nsel + 8 * B * Lq * k, "macs": 0.0}
+    if Lq == 1:  # decode runs the fused indexer -> top-k: one stage, the two stages' work
+        return {"indexer_topk": {"bytes": ix["bytes"] + tk["bytes"], "macs": ix["macs"]}, "sparse_mla": ml,
+                "indexer_kl": kl}
     return {"indexer": ix, "topk": tk, "sparse_mla": ml, "indexer_kl": kl}
 
 
@@ -150,7 +153,7 @@ def tensor_peak(stage, peaks, sustained):
     """Dense tensor peak (TFLOP/s) of a stage's contraction: bf16 for attention, FP8 (the bf16
     measurement times the datasheet's FP8/bf16 ratio) for the indexer; None for the rest."""
     bf16 = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
-    if stage == "indexer":
+    if stage in ("indexer", "indexer_topk"):
         return FP8_OVER_BF16 * bf16
     if stage in ("sparse_mla", "dense_mla"):
         return bf16
@@ -315,6 +318,7 @@ class Step:
         self.p = torch.empty(B, Lq, pk, dtype=torch.float32, device=device) if wl.emit_p else None
         self.loss = torch.empty(1, dtype=torch.float32, device=device)
         nws = max(dsa.dsa_workspace_bytes(dsa.DSA_OP_SPARSE_MLA_FWD, B, Lq, Lk, wl.k, wl.H),
+                  dsa.dsa_workspace_bytes(dsa.DSA_OP_INDEXER_TOPK, B, Lq, Lk, wl.k, 0),
                   dsa.dsa_workspace_bytes(dsa.DSA_OP_DENSE_MLA_FWD, B, Lq, Lk, 0, wl.H) if wl.dense else 0,
                   dsa.dsa_workspace_bytes(dsa.DSA_OP_INDEXER_KL, B, Lq, Lk, wl.k, 0), 16)
         self.ws = torch.empty(nws, dtype=torch.uint8, device=device)
@@ -340,6 +344,16 @@ class Step:
         dsa, d, wl = self.dsa, self.d, self.wl
         if ev:
             ev[0].record()
+        if wl.Lq == 1 and not wl.dense:  # decode: the fused indexer -> top-k (one stage)
+            dsa.dsa_indexer_topk(d["qI"], d["kI"], d["w"], self.scores, self.idx, self.ws)
+            if ev:
+                ev[1].record()
+                ev[2].record()
+            dsa.dsa_sparse_mla_fwd(d["q"], d["kv"], self.idx, wl.scale, self.out, self.lse, self.p, self.ws)
+            if ev:
+                ev[3].record()
+                ev[4].record()
+            return
         dsa.dsa_indexer(d["qI"], d["kI"], d["w"], self.scores)
         if ev:
             ev[1].record()
@@ -456,6 +470,9 @@ def measure(shard, device, steps, warmup, world, peaks, e2e=True):
         stage_ms[attn].append(e[2].elapsed_time(e[3]))
         stage_ms["indexer_kl"].append(e[3].elapsed_time(e[4]))
     if wl.dense:
+        del stage_ms["topk"]
+    if wl.Lq == 1 and not wl.dense:  # the fused decode call: indexer and top-k are one stage
+        stage_ms["indexer_topk"] = stage_ms.pop("indexer")
         del stage_ms["topk"]
     total_ms = max_over_ranks(sum(step_ms), device)  # the slowest rank's time
     ms_per_step = total_ms / steps

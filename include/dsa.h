@@ -58,7 +58,8 @@ enum {
   DSA_OP_SPARSE_MLA_FWD = 2,
   DSA_OP_INDEXER_KL = 3,
   DSA_OP_DENSE_MLA_FWD = 4,
-  DSA_OP_INDEXER_KL_DENSE = 5
+  DSA_OP_INDEXER_KL_DENSE = 5,
+  DSA_OP_INDEXER_TOPK = 6
 };
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -102,6 +103,22 @@ dsa_status dsa_indexer(const void* q_fp8, const void* k_fp8, const float* w, flo
  */
 dsa_status dsa_topk(const float* scores, int32_t* idx, int B, int Lq, int Lk, int k, void* ws,
                     size_t ws_bytes, dsa_stream_t stream);
+
+/*
+ * Indexer and top-k in one call: dsa_indexer followed by dsa_topk, with identical results
+ * (scores and idx as those two entry points define them).  For decode (Lq == 1, (H_I, d_I) in
+ * {(64, 128), (32, 128)}) the two are fused: the indexer's epilogue also counts each row's
+ * visible scores by the top-k's first radix digit, so the selection starts from that histogram
+ * instead of counting the row itself (the "fused top-k" the "DeepSeek-V3.2" analysis page names
+ * among the indexer's constant-factor savings, sec. 5.2 closing paragraph; decode step cost of
+ * sec. 5.3, eq. (23)).
+ *   ws: dsa_workspace_bytes(DSA_OP_INDEXER_TOPK, B, Lq, Lk, k, 0) bytes (the per-row histograms,
+ *       B * Lq * 8 KiB for decode, 0 otherwise); it is cleared on the stream by the call itself.
+ * Supported: the union of dsa_indexer's and dsa_topk's limits.
+ */
+dsa_status dsa_indexer_topk(const void* q_fp8, const void* k_fp8, const float* w, float* scores,
+                            int32_t* idx, int B, int Lq, int Lk, int H_I, int d_I, int k, void* ws,
+                            size_t ws_bytes, dsa_stream_t stream);
 
 /*
  * Sparse attention in MLA's MQA mode over the selected latents ("DeepSeek-V3.2" analysis

@@ -19,17 +19,17 @@ __all__ = [
     "DsaError", "load", "dsa_status_str", "dsa_version", "dsa_workspace_bytes", "dsa_indexer",
     "dsa_topk", "dsa_sparse_mla_fwd", "dsa_indexer_kl", "dsa_indexer_kl_noalloc",
     "dsa_last_device_status", "dsa_set_wait_limit_ns", "dsa_selftest_wait", "dsa_dense_mla_fwd",
-    "dsa_indexer_kl_dense",
+    "dsa_indexer_kl_dense", "dsa_indexer_topk",
     "DSA_OP_INDEXER", "DSA_OP_TOPK", "DSA_OP_SPARSE_MLA_FWD", "DSA_OP_INDEXER_KL",
-    "DSA_OP_DENSE_MLA_FWD", "DSA_OP_INDEXER_KL_DENSE", "EXPORTED",
+    "DSA_OP_DENSE_MLA_FWD", "DSA_OP_INDEXER_KL_DENSE", "DSA_OP_INDEXER_TOPK", "EXPORTED",
 ]
 
 DSA_OP_INDEXER, DSA_OP_TOPK, DSA_OP_SPARSE_MLA_FWD, DSA_OP_INDEXER_KL = 0, 1, 2, 3
-DSA_OP_DENSE_MLA_FWD, DSA_OP_INDEXER_KL_DENSE = 4, 5
+DSA_OP_DENSE_MLA_FWD, DSA_OP_INDEXER_KL_DENSE, DSA_OP_INDEXER_TOPK = 4, 5, 6
 EXPORTED = ("dsa_status_str", "dsa_version", "dsa_workspace_bytes", "dsa_indexer", "dsa_topk",
             "dsa_sparse_mla_fwd", "dsa_indexer_kl", "dsa_indexer_kl_noalloc",
             "dsa_last_device_status", "dsa_set_wait_limit_ns", "dsa_selftest_wait",
-            "dsa_dense_mla_fwd", "dsa_indexer_kl_dense")
+            "dsa_dense_mla_fwd", "dsa_indexer_kl_dense", "dsa_indexer_topk")
 
 
 class DsaError(RuntimeError):
@@ -66,9 +66,10 @@ def load(rebuild: bool = False) -> ctypes.CDLL:
         lib.dsa_selftest_wait.argtypes = [vp]
         lib.dsa_dense_mla_fwd.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, f32, vp, vp, vp, vp, sz, vp]
         lib.dsa_indexer_kl_dense.argtypes = [vp, vp, i32, i32, i32, vp, vp, vp, sz, vp]
+        lib.dsa_indexer_topk.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, sz, vp]
         for name in ("dsa_indexer", "dsa_topk", "dsa_sparse_mla_fwd", "dsa_indexer_kl",
                      "dsa_indexer_kl_noalloc", "dsa_last_device_status", "dsa_set_wait_limit_ns",
-                     "dsa_selftest_wait", "dsa_dense_mla_fwd", "dsa_indexer_kl_dense"):
+                     "dsa_selftest_wait", "dsa_dense_mla_fwd", "dsa_indexer_kl_dense", "dsa_indexer_topk"):
             getattr(lib, name).restype = i32
         _lib = lib
     return _lib
@@ -144,6 +145,24 @@ def dsa_topk(scores: torch.Tensor, idx: torch.Tensor, stream=None) -> None:
     _check(idx, "idx", torch.int32, (B, Lq, k))
     _raise("dsa_topk", load().dsa_topk(_ptr(scores), _ptr(idx), B, Lq, Lk, k, None, 0,
                                        _stream(stream)))
+
+
+def dsa_indexer_topk(q_fp8: torch.Tensor, k_fp8: torch.Tensor, w: torch.Tensor, scores: torch.Tensor,
+                     idx: torch.Tensor, ws: torch.Tensor | None = None, stream=None) -> None:
+    """dsa_indexer then dsa_topk in one call (fused for decode: the indexer counts the top-k's
+    first radix digit); ws: dsa_workspace_bytes(DSA_OP_INDEXER_TOPK, ...) bytes."""
+    B, Lq, H_I, d_I = q_fp8.shape
+    Lk = k_fp8.shape[1]
+    k = idx.shape[2]
+    _check(q_fp8, "q_fp8", torch.float8_e4m3fn, (B, Lq, H_I, d_I))
+    _check(k_fp8, "k_fp8", torch.float8_e4m3fn, (B, Lk, d_I))
+    _check(w, "w", torch.float32, (B, Lq, H_I))
+    _check(scores, "scores", torch.float32, (B, Lq, Lk))
+    _check(idx, "idx", torch.int32, (B, Lq, k))
+    wsp, wsb = _ws(ws)
+    _raise("dsa_indexer_topk",
+           load().dsa_indexer_topk(_ptr(q_fp8), _ptr(k_fp8), _ptr(w), _ptr(scores), _ptr(idx), B, Lq, Lk, H_I,
+                                   d_I, k, wsp, wsb, _stream(stream)))
 
 
 def dsa_sparse_mla_fwd(q: torch.Tensor, kv: torch.Tensor, idx: torch.Tensor, scale: float,

@@ -138,7 +138,7 @@ dsa_status launch(void (*kern)(KArgs...), unsigned grid, unsigned block, size_t 
 // ------------------------------------------------------------------------------ indexer
 template <int H_I, int D_I, int G>
 dsa_status launch_indexer(const void* q, const void* kk, const float* w, float* scores, int B,
-                          int Lq, int Lk, int sms, cudaStream_t stream) {
+                          int Lq, int Lk, int sms, cudaStream_t stream, uint32_t* hist = nullptr) {
   using Cfg = dsa::indexer::Cfg<H_I, D_I, G>;
   const CUtensorMapSwizzle swz = D_I == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
                                  : D_I == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
@@ -154,6 +154,7 @@ dsa_status launch_indexer(const void* q, const void* kk, const float* w, float* 
   p.k = static_cast<const uint8_t*>(kk);
   p.w = w;
   p.scores = scores;
+  p.hist = hist;
   p.B = B;
   p.Lq = Lq;
   p.Lk = Lk;
@@ -183,13 +184,13 @@ dsa_status launch_indexer(const void* q, const void* kk, const float* w, float* 
 // ------------------------------------------------------------------------------ top-k
 template <int C, int KPT>
 dsa_status launch_topk(const float* scores, int32_t* idx, int B, int Lq, int Lk, int k,
-                       cudaStream_t stream) {
+                       cudaStream_t stream, const uint32_t* ghist) {
   auto kern = dsa::topk::topk_kernel<C, KPT>;
   constexpr int smem = dsa::topk::dyn_smem_bytes<KPT>();
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return DSA_ERR_CUDA;
   return launch(kern, static_cast<unsigned>(B) * Lq * C, dsa::topk::kThreads, smem, stream, C, scores, idx, B, Lq,
-                Lk, k);
+                Lk, k, ghist);
 }
 
 // Keys per CTA for a row split over c CTAs (a multiple of 4, as the kernel computes it).
@@ -205,12 +206,45 @@ int topk_cluster_size(int rows, int Lk, int sms) {
 
 template <int C>
 dsa_status launch_topk_c(const float* scores, int32_t* idx, int B, int Lq, int Lk, int k,
-                         cudaStream_t st) {
+                         cudaStream_t st, const uint32_t* ghist) {
   const int slice = topk_slice(Lk, C);
-  if (slice <= 4 * dsa::topk::kThreads) return launch_topk<C, 4>(scores, idx, B, Lq, Lk, k, st);
-  if (slice <= 8 * dsa::topk::kThreads) return launch_topk<C, 8>(scores, idx, B, Lq, Lk, k, st);
-  if (slice <= 16 * dsa::topk::kThreads) return launch_topk<C, 16>(scores, idx, B, Lq, Lk, k, st);
-  return launch_topk<C, 32>(scores, idx, B, Lq, Lk, k, st);
+  if (slice <= 4 * dsa::topk::kThreads) return launch_topk<C, 4>(scores, idx, B, Lq, Lk, k, st, ghist);
+  if (slice <= 8 * dsa::topk::kThreads) return launch_topk<C, 8>(scores, idx, B, Lq, Lk, k, st, ghist);
+  if (slice <= 16 * dsa::topk::kThreads) return launch_topk<C, 16>(scores, idx, B, Lq, Lk, k, st, ghist);
+  return launch_topk<C, 32>(scores, idx, B, Lq, Lk, k, st, ghist);
+}
+
+// Top-k with the validated sizes; ghist (nullable) holds each row's top-digit counts.
+dsa_status run_topk(const float* scores, int32_t* idx, int B, int Lq, int Lk, int k, int sms, cudaStream_t st,
+                    const uint32_t* ghist) {
+  switch (topk_cluster_size(B * Lq, Lk, sms)) {
+    case 1: return launch_topk_c<1>(scores, idx, B, Lq, Lk, k, st, ghist);
+    case 2: return launch_topk_c<2>(scores, idx, B, Lq, Lk, k, st, ghist);
+    case 4: return launch_topk_c<4>(scores, idx, B, Lq, Lk, k, st, ghist);
+    default: return launch_topk_c<8>(scores, idx, B, Lq, Lk, k, st, ghist);
+  }
+}
+
+// Indexer with the validated sizes.  hist (nullable, decode kernels only) receives each row's
+// top-digit counts; returns DSA_ERR_UNSUPPORTED for shapes outside the compiled kernels.
+dsa_status run_indexer(const void* q_fp8, const void* k_fp8, const float* w, float* scores, int B, int Lq, int Lk,
+                       int H_I, int d_I, int sms, cudaStream_t st, uint32_t* hist) {
+  const bool decode = (Lq == 1);
+  if (H_I == 64 && d_I == 128)
+    return decode ? launch_indexer<64, 128, 1>(q_fp8, k_fp8, w, scores, B, Lq, Lk, sms, st, hist)
+                  : launch_indexer<64, 128, 4>(q_fp8, k_fp8, w, scores, B, Lq, Lk, sms, st);
+  if (H_I == 32 && d_I == 128)
+    return decode ? launch_indexer<32, 128, 1>(q_fp8, k_fp8, w, scores, B, Lq, Lk, sms, st, hist)
+                  : launch_indexer<32, 128, 8>(q_fp8, k_fp8, w, scores, B, Lq, Lk, sms, st);
+  if (H_I == 16 && d_I == 128) return launch_indexer<16, 128, 16>(q_fp8, k_fp8, w, scores, B, Lq, Lk, sms, st);
+  if (H_I == 8 && d_I == 64) return launch_indexer<8, 64, 32>(q_fp8, k_fp8, w, scores, B, Lq, Lk, sms, st);
+  if (H_I == 4 && d_I == 32) return launch_indexer<4, 32, 64>(q_fp8, k_fp8, w, scores, B, Lq, Lk, sms, st);
+  return DSA_ERR_UNSUPPORTED;
+}
+
+// Whether the indexer of this shape has the decode kernel that counts top digits.
+inline bool fused_topk_shape(int Lq, int H_I, int d_I) {
+  return Lq == 1 && d_I == 128 && (H_I == 64 || H_I == 32);
 }
 
 // ------------------------------------------------------------------------------ sparse MLA
@@ -400,6 +434,9 @@ size_t dsa_workspace_bytes(int op, int B, int Lq, int Lk, int k, int H) {
       return std::max(mla_ws_bytes(static_cast<int>(rows), Lk, H, 512, sms),
                       mla_ws_bytes(static_cast<int>(rows), Lk, H, 64, sms));
     }
+    case DSA_OP_INDEXER_TOPK:
+      // the decode kernels' top-digit histograms (no workspace for other shapes)
+      return Lq == 1 ? static_cast<size_t>(rows) * 2048 * sizeof(uint32_t) : 0;
     case DSA_OP_INDEXER_KL:
     case DSA_OP_INDEXER_KL_DENSE:
       return static_cast<size_t>(rows) * sizeof(float);
@@ -422,21 +459,8 @@ dsa_status dsa_indexer(const void* q_fp8, const void* k_fp8, const float* w, flo
   DeviceInfo dev;
   const dsa_status ds = current_device(dev);
   if (ds != DSA_OK) return ds;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const bool decode = (Lq == 1);
-  if (H_I == 64 && d_I == 128)
-    return decode ? launch_indexer<64, 128, 1>(q_fp8, k_fp8, w, scores, B, Lq, Lk, dev.sms, st)
-                  : launch_indexer<64, 128, 4>(q_fp8, k_fp8, w, scores, B, Lq, Lk, dev.sms, st);
-  if (H_I == 32 && d_I == 128)
-    return decode ? launch_indexer<32, 128, 1>(q_fp8, k_fp8, w, scores, B, Lq, Lk, dev.sms, st)
-                  : launch_indexer<32, 128, 8>(q_fp8, k_fp8, w, scores, B, Lq, Lk, dev.sms, st);
-  if (H_I == 16 && d_I == 128)
-    return launch_indexer<16, 128, 16>(q_fp8, k_fp8, w, scores, B, Lq, Lk, dev.sms, st);
-  if (H_I == 8 && d_I == 64)
-    return launch_indexer<8, 64, 32>(q_fp8, k_fp8, w, scores, B, Lq, Lk, dev.sms, st);
-  if (H_I == 4 && d_I == 32)
-    return launch_indexer<4, 32, 64>(q_fp8, k_fp8, w, scores, B, Lq, Lk, dev.sms, st);
-  return DSA_ERR_UNSUPPORTED;
+  return run_indexer(q_fp8, k_fp8, w, scores, B, Lq, Lk, H_I, d_I, dev.sms, static_cast<cudaStream_t>(stream),
+                     nullptr);
 }
 
 dsa_status dsa_topk(const float* scores, int32_t* idx, int B, int Lq, int Lk, int k, void* ws,
@@ -451,13 +475,32 @@ dsa_status dsa_topk(const float* scores, int32_t* idx, int B, int Lq, int Lk, in
   DeviceInfo dev;
   const dsa_status ds = current_device(dev);
   if (ds != DSA_OK) return ds;
+  return run_topk(scores, idx, B, Lq, Lk, k, dev.sms, static_cast<cudaStream_t>(stream), nullptr);
+}
+
+dsa_status dsa_indexer_topk(const void* q_fp8, const void* k_fp8, const float* w, float* scores, int32_t* idx,
+                            int B, int Lq, int Lk, int H_I, int d_I, int k, void* ws, size_t ws_bytes,
+                            dsa_stream_t stream) {
+  if (!q_fp8 || !k_fp8 || !w || !scores || !idx) return DSA_ERR_INVALID_ARG;
+  if (B <= 0 || Lq <= 0 || Lk <= 0 || Lq > Lk || H_I <= 0 || d_I <= 0 || k <= 0) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q_fp8) || !aligned16(k_fp8) || !aligned16(w) || !aligned16(scores) || !aligned16(idx))
+    return DSA_ERR_INVALID_ARG;
+  if (static_cast<long>(B) * Lk > INT32_MAX || static_cast<long>(B) * Lq * H_I > INT32_MAX)
+    return DSA_ERR_UNSUPPORTED;
+  if (k > 4096 || topk_slice(Lk, 8) > dsa::topk::kMaxSlice) return DSA_ERR_UNSUPPORTED;
+  if (static_cast<long>(B) * Lq * 8 > INT32_MAX) return DSA_ERR_UNSUPPORTED;
+  const bool fused = fused_topk_shape(Lq, H_I, d_I);
+  const size_t need = fused ? static_cast<size_t>(B) * Lq * 2048 * sizeof(uint32_t) : 0;
+  if (fused && (ws == nullptr || ws_bytes < need || !aligned16(ws))) return DSA_ERR_INVALID_ARG;
+  DeviceInfo dev;
+  const dsa_status ds = current_device(dev);
+  if (ds != DSA_OK) return ds;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  switch (topk_cluster_size(B * Lq, Lk, dev.sms)) {
-    case 1: return launch_topk_c<1>(scores, idx, B, Lq, Lk, k, st);
-    case 2: return launch_topk_c<2>(scores, idx, B, Lq, Lk, k, st);
-    case 4: return launch_topk_c<4>(scores, idx, B, Lq, Lk, k, st);
-    default: return launch_topk_c<8>(scores, idx, B, Lq, Lk, k, st);
-  }
+  uint32_t* hist = fused ? static_cast<uint32_t*>(ws) : nullptr;
+  if (fused && cudaMemsetAsync(hist, 0, need, st) != cudaSuccess) return DSA_ERR_CUDA;
+  const dsa_status si = run_indexer(q_fp8, k_fp8, w, scores, B, Lq, Lk, H_I, d_I, dev.sms, st, hist);
+  if (si != DSA_OK) return si;
+  return run_topk(scores, idx, B, Lq, Lk, k, dev.sms, st, hist);
 }
 
 dsa_status dsa_sparse_mla_fwd(const void* q_bf16, const void* kv_bf16, const int32_t* idx, int B,

@@ -9,13 +9,17 @@
 // Persistent, warp-specialised CTA (one per SM):
 //   warp 0        TMA producer: the q_I group once per work item, then k_I tiles (12 stages
 //                 for decode, 6 otherwise).  For decode (one query per tile, a pure stream of
-//                 k_I) warps 0, 2 and 3 load the k_I tiles with 16-byte cp.async copies written
-//                 straight into the 128B-swizzled layout instead: plain loads stream from HBM
-//                 faster than TMA tile copies on B200 (about 6.0 against 5.5 TB/s for a 512 MiB
-//                 read), and decode is bound by that stream.
+//                 k_I) warps 0 and 2 load the k_I tiles with 16-byte cp.async copies written
+//                 straight into the 128B-swizzled layout instead, and warp 3 loads the q_I
+//                 groups: plain loads stream from HBM faster than TMA tile copies on B200 (about
+//                 6.0 against 5.5 TB/s for a 512 MiB read), and decode is bound by that stream.
 //   warp 1        MMA issuer (one thread): d_I/32 MMAs of 128 x N x 32 per tile
 //   warp 2        TMEM allocator (2 accumulators of N columns, double-buffered)
-//   warps 4..11   epilogue: tcgen05.ld -> ReLU * w -> head sum -> mask -> store
+//   warps 4..11   epilogue: tcgen05.ld -> ReLU * w -> head sum -> mask -> store; for decode
+//                 with a `hist` buffer (the fused indexer -> top-k path) it also counts every
+//                 visible score of the row by the top 11 bits of its order-preserving key, the
+//                 top-k's first radix digit (shared-memory counts per work item, added to the
+//                 row's global histogram at the item's end).
 // Work item = (sequence, group of G queries, chunk of key tiles); key tiles beyond the
 // group's last visible position skip the MMA and are written as -inf directly.
 #pragma once
@@ -35,6 +39,7 @@ struct Params {
   const uint8_t* k;  // k_I [B * Lk, d_I] (the decode loads read it directly)
   const float* w;
   float* scores;
+  uint32_t* hist;    // nullable, decode only: [B * Lq][2048] counts of the scores' top digit
   int B, Lq, Lk;
   int n_qg;   // query groups per sequence
   int n_kt;   // key tiles per sequence
@@ -43,9 +48,9 @@ struct Params {
   int n_items;
 };
 
-// Decode k_I producers (cp.async): warps 0, 2 and 3, and how many tiles each keeps in flight
+// Decode k_I producers (cp.async): warps 0 and 2, and how many tiles each keeps in flight
 // before it signals the oldest one.
-constexpr int kLoadThreads = 96;
+constexpr int kLoadThreads = 64;
 constexpr int kLoadLag = 6;
 
 template <int H_I, int D_I, int G>
@@ -70,7 +75,8 @@ struct Cfg {
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kOffQ + 2 * ((kQBytes + 1023) / 1024) * 1024;
   static constexpr int kOffW = kOffK + kStages * kKBytes;
-  static constexpr int kOffBar = kOffW + 2 * N * 4;
+  static constexpr int kOffHist = kOffW + 2 * N * 4;                 // decode: [2048] digit counts
+  static constexpr int kOffBar = kOffHist + (G == 1 ? 2048 * 4 : 0);
   static constexpr int kNumBars = 2 * kStages + 8;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
@@ -115,6 +121,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sQ = smem + C::kOffQ;
   uint8_t* sK = smem + C::kOffK;
   float* sW = reinterpret_cast<float*>(smem + C::kOffW);
+  uint32_t* sHist = reinterpret_cast<uint32_t*>(smem + C::kOffHist);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
   uint64_t* k_full = bars;
   uint64_t* k_empty = bars + C::kStages;
@@ -151,39 +158,50 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
   pdl_wait();  // first global access below
 
-  if (C::kCpAsyncK && (warp == 0 || warp == 2 || warp == 3)) {
-    // ------------------------------------------------------------------ decode producer
-    // Lane 0 of warp 0 loads each item's q_I group by TMA; the 96 threads load the k_I tiles:
-    // thread pt copies the 16-byte chunks pt, pt + 96, ... of a tile (consecutive threads read
-    // consecutive bytes), each to its 128B-swizzled place.  A thread signals tile j on the
-    // tile's barrier once its copies of tile j have landed (cp.async.wait_group) and are made
-    // visible to the tensor cores' async proxy, which it checks after issuing tile j + lag;
-    // tile j + kStages waits for tile j to be consumed, which needs j signalled (lag < stages).
-    const int pt = (warp == 0 ? 0 : warp - 1) * 32 + lane;
+  if (C::kCpAsyncK && warp == 3) {
+    // ------------------------------------------------------------------ decode: q_I groups
+    // A thread of its own: its wait for a free q_I buffer (item u - 2 consumed) must never hold
+    // back the k_I producers, which signal their tiles a few tiles late.
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      int qi = 0;
+      for (int u = blockIdx.x; u < p.n_items; u += gridDim.x) {
+        int b, qg, kc, kt0, kt1, n_comp;
+        decode_item(p, u, b, qg, kc);
+        item_tiles<G>(p, qg, kc, kt0, kt1, n_comp);
+        if (n_comp == 0) continue;
+        const int qb = qi & 1;
+        const uint32_t qph = (qi >> 1) & 1;
+        if (!mbar_wait(&q_empty[qb], qph ^ 1, abort_flag, 1)) break;
+        mbar_arrive_expect_tx(&q_full[qb], C::kQBytes);
+        tma_load_2d(sQ + qb * ((C::kQBytes + 1023) / 1024) * 1024, &tm_q, &q_full[qb], 0,
+                    (b * p.Lq + qg * G) * H_I);
+        ++qi;
+      }
+    }
+  } else if (C::kCpAsyncK && (warp == 0 || warp == 2)) {
+    // ------------------------------------------------------------------ decode: k_I tiles
+    // Thread pt of the 64 copies the 16-byte chunks pt, pt + 64, ... of a tile (consecutive
+    // threads read consecutive bytes), each to its 128B-swizzled place.  A thread signals tile
+    // j on the tile's barrier once its copies of tile j have landed (cp.async.wait_group) and are
+    // made visible to the tensor cores' async proxy, which it checks after issuing tile j + lag.
+    // No wait of these threads depends on a tile they have not signalled: tile j + kStages
+    // waits for tile j to be consumed, which needs only tiles <= j signalled (lag < stages) and
+    // the q_I group of tile j's item, loaded by warp 3 once the item two back is consumed.
+    const int pt = (warp == 0 ? 0 : 32) + lane;
     const size_t k_rows = static_cast<size_t>(p.B) * p.Lk;
+    // k_I is read once: its lines go first out of L2, so that the scores written meanwhile stay
+    // there for the top-k that reads them next
+    const uint64_t evict_first = l2_evict_first_policy();
     int ks = 0, sig = 0;  // stage of the next tile; stage of the oldest unsignalled tile
     uint32_t kph = 0;
     int pending = 0;      // tiles issued but not signalled by this thread
-    int qi = 0;
     bool ok = true;
-    if (warp == 0 && lane == 0) tma_prefetch_desc(&tm_q);
     for (int u = blockIdx.x; ok && u < p.n_items; u += gridDim.x) {
       int b, qg, kc, kt0, kt1, n_comp;
       decode_item(p, u, b, qg, kc);
       item_tiles<G>(p, qg, kc, kt0, kt1, n_comp);
-      if (n_comp == 0) continue;
-      if (warp == 0 && lane == 0) {
-        const int qb = qi & 1;
-        const uint32_t qph = (qi >> 1) & 1;
-        if (!mbar_wait(&q_empty[qb], qph ^ 1, abort_flag, 1)) ok = false;
-        if (ok) {
-          mbar_arrive_expect_tx(&q_full[qb], C::kQBytes);
-          tma_load_2d(sQ + qb * ((C::kQBytes + 1023) / 1024) * 1024, &tm_q, &q_full[qb], 0,
-                      (b * p.Lq + qg * G) * H_I);
-        }
-      }
-      ++qi;
-      for (int tt = 0; ok && tt < n_comp; ++tt) {
+      for (int tt = 0; tt < n_comp; ++tt) {
         if (!mbar_wait(&k_empty[ks], kph ^ 1, abort_flag, 2)) {
           ok = false;
           break;
@@ -193,7 +211,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = pt; c < kTileKeys * (D_I / 16); c += kLoadThreads) {
           const int r = c >> 3, ch = c & 7;
           const bool valid = row0 + r < k_rows;  // rows past the tensor are zero-filled
-          cp_async_16(dst + swizzled_offset(r, ch, 128), p.k + (valid ? (row0 + r) * D_I + ch * 16 : 0), valid);
+          cp_async_16_hint(dst + swizzled_offset(r, ch, 128), p.k + (valid ? (row0 + r) * D_I + ch * 16 : 0), valid,
+                           evict_first);
         }
         cp_async_commit();
         if (++pending > kLoadLag) {
@@ -301,6 +320,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     int gt = 0;  // tiles with an MMA seen so far, over all items (both groups count every one)
     int it = 0;
+    const bool count = (G == 1) && p.hist != nullptr;
+    if (count)
+      for (int x = e; x < 2048; x += 256) sHist[x] = 0u;  // ordered by the item's first barrier
     for (int u = blockIdx.x; u < p.n_items; u += gridDim.x, ++it) {
       int b, qg, kc, kt0, kt1, n_comp;
       decode_item(p, u, b, qg, kc);
@@ -349,7 +371,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (i < p.Lq) {
               const int t = i + p.Lk - p.Lq;
               p.scores[(row_base + i) * p.Lk + s] = (s <= t) ? acc[g] : -INFINITY;
+              if (G == 1 && count && s <= t) atomicAdd(&sHist[ordered_key(acc[g]) >> 21], 1u);
             }
+          }
+        }
+      }
+      if (count) {  // this item's counts into the row's histogram; the next item starts from zero
+        named_bar_sync(2, 256);
+        uint32_t* gh = p.hist + (row_base + i0) * 2048;
+        for (int x = e; x < 2048; x += 256) {
+          const uint32_t v = sHist[x];
+          if (v) {
+            atomicAdd(gh + x, v);
+            sHist[x] = 0u;
           }
         }
       }

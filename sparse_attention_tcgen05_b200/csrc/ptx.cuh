@@ -279,6 +279,30 @@ template <int N>
 __device__ __forceinline__ void cp_async_wait_group() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
+// An L2 policy that evicts first the lines it is attached to (for a stream read once, so that
+// it does not push out data that is read again soon).
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+// cp_async_16 with an L2 cache policy for the source lines.
+__device__ __forceinline__ void cp_async_16_hint(uint32_t smem_dst, const void* src, bool valid, uint64_t policy) {
+  const uint32_t src_bytes = valid ? 16u : 0u;
+  asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2, %3;" ::"r"(smem_dst), "l"(src),
+               "r"(src_bytes), "l"(policy)
+               : "memory");
+}
+
+// Order-preserving 32-bit key of an fp32 score: a > b as floats iff key(a) > key(b) as
+// unsigned integers, with -0 folded onto +0.  Every finite or infinite score maps to a key
+// >= 0x007FFFFF, so 0 can mark an empty slot.  The top-k's radix digits are bits of this key.
+__device__ __forceinline__ uint32_t ordered_key(float f) {
+  uint32_t u = __float_as_uint(f);
+  if (u == 0x80000000u) u = 0u;  // -0 ties with +0
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
 // Arrive on `bar` once all of this thread's prior cp.async copies have landed
 // (the arrival counts toward the barrier's expected count).
 __device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {

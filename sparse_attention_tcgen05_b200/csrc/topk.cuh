@@ -6,7 +6,9 @@
 // 32-bit keys (read from HBM once).  The k-th largest key T is found by radix select on digits
 // of 11, 11 and 10 bits:
 //   1. every CTA counts its keys by the top digit; the cluster's counts (summed through
-//      distributed shared memory, two bins per request) give the digit d1 that holds T;
+//      distributed shared memory, two bins per request) give the digit d1 that holds T.  When
+//      the indexer already counted the row's top digits (the fused decode path, `ghist`), that
+//      histogram gives d1 directly and this pass and its cluster round are skipped;
 //   2. the candidates - keys whose top digit is d1, usually a few thousand per row - are pushed
 //      with their positions into every CTA of the cluster, together with each CTA's count of
 //      keys above d1; after one cluster barrier every CTA settles the two lower digits on the
@@ -37,14 +39,6 @@ template <int KPT>
 __host__ __device__ constexpr int stage_bytes() { return kThreads * KPT * 4; }
 template <int KPT>
 __host__ __device__ constexpr int dyn_smem_bytes() { return stage_bytes<KPT>() + kCandBytes; }
-
-// Every finite or infinite score maps to a key >= 0x007FFFFF; 0 marks an empty register slot
-// and can never be selected (at least k real keys exist whenever a row is selected).
-__device__ __forceinline__ uint32_t ordered_key(float f) {
-  uint32_t u = __float_as_uint(f);
-  if (u == 0x80000000u) u = 0u;  // -0 ties with +0
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
 
 __device__ __forceinline__ uint32_t ld_peer_u32(const uint32_t* local, uint32_t rank) {
   uint32_t v;
@@ -211,7 +205,7 @@ __device__ __forceinline__ uint2 block_exclusive2(uint32_t a, uint32_t b, uint32
 template <int C, int KPT>
 __global__ void __launch_bounds__(kThreads, 1)
     topk_kernel(const float* __restrict__ scores, int32_t* __restrict__ idx, int B, int Lq, int Lk,
-                int k) {
+                int k, const uint32_t* __restrict__ ghist) {
   static_assert(KPT == 4 || KPT == 8 || KPT == 16 || KPT == 32, "keys per thread");
   static_assert(C == 1 || C == 2 || C == 4 || C == kMaxCluster, "cluster size");
   constexpr int kCpr = KPT / 4;  // chunks per thread
@@ -264,6 +258,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     hist[1][x] = 0u;
   }
   __syncthreads();
+  // With the indexer's histogram no cluster round precedes the candidate push, so every CTA's
+  // n_cand must be zero before any peer reserves room in it: one cluster barrier here, which
+  // overlaps the previous kernel's tail.
+  const bool pre = ghist != nullptr;
+  if (C > 1 && pre) cluster_barrier();
   pdl_wait();  // the scores are written by the previous kernel
   if (tid == 0 && nbulk > 0u) {
     mbar_arrive_expect_tx(&load_bar, nbulk);
@@ -298,15 +297,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint4 q = make_uint4(x < cnt ? ordered_key(f.x) : 0u, x + 1 < cnt ? ordered_key(f.y) : 0u,
                                x + 2 < cnt ? ordered_key(f.z) : 0u, x + 3 < cnt ? ordered_key(f.w) : 0u);
     stk[g] = q;
-    if (q.x) atomicAdd(&hist[0][q.x >> 21], 1u);
-    if (q.y) atomicAdd(&hist[0][q.y >> 21], 1u);
-    if (q.z) atomicAdd(&hist[0][q.z >> 21], 1u);
-    if (q.w) atomicAdd(&hist[0][q.w >> 21], 1u);
+    if (!pre) {
+      if (q.x) atomicAdd(&hist[0][q.x >> 21], 1u);
+      if (q.y) atomicAdd(&hist[0][q.y >> 21], 1u);
+      if (q.z) atomicAdd(&hist[0][q.z >> 21], 1u);
+      if (q.w) atomicAdd(&hist[0][q.w >> 21], 1u);
+    }
   }
   __syncthreads();
-  if (C > 1) cluster_barrier();  // every CTA's counts are complete and its n_cand is zero
   uint32_t d1, k1;
-  select_digit<C>(hist[0], 2048, static_cast<uint32_t>(k), scan, result, d1, k1);
+  if (pre) {  // the whole row's top-digit counts, from the indexer
+    select_digit<1>(ghist + static_cast<size_t>(row) * 2048, 2048, static_cast<uint32_t>(k), scan, result, d1, k1);
+  } else {
+    if (C > 1) cluster_barrier();  // every CTA's counts are complete and its n_cand is zero
+    select_digit<C>(hist[0], 2048, static_cast<uint32_t>(k), scan, result, d1, k1);
+  }
 
   // ---- the candidates (keys in digit d1) with their positions, into every CTA's buffer
   uint2* cand = reinterpret_cast<uint2*>(dyn + stage_bytes<KPT>());

@@ -106,10 +106,14 @@ def run_path(dw: DeviceWorkload, emit_p: bool | None = None):
     out = torch.empty(wl.B, wl.Lq, wl.H, wl.d_v, dtype=torch.bfloat16, device=dev)
     lse = torch.empty(wl.B, wl.Lq, wl.H, dtype=torch.float32, device=dev)
     p_sel = torch.empty(wl.B, wl.Lq, wl.k, dtype=torch.float32, device=dev) if emit_p else None
-    ws_bytes = dsa.dsa_workspace_bytes(dsa.DSA_OP_SPARSE_MLA_FWD, wl.B, wl.Lq, wl.Lk, wl.k, wl.H)
+    ws_bytes = max(dsa.dsa_workspace_bytes(dsa.DSA_OP_SPARSE_MLA_FWD, wl.B, wl.Lq, wl.Lk, wl.k, wl.H),
+                   dsa.dsa_workspace_bytes(dsa.DSA_OP_INDEXER_TOPK, wl.B, wl.Lq, wl.Lk, wl.k, 0))
     ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
-    dsa.dsa_indexer(dw.qI, dw.kI, dw.w, scores)
-    dsa.dsa_topk(scores, idx)
+    if wl.Lq == 1:  # decode: the fused indexer -> top-k entry point, as the bench runs it
+        dsa.dsa_indexer_topk(dw.qI, dw.kI, dw.w, scores, idx, ws)
+    else:
+        dsa.dsa_indexer(dw.qI, dw.kI, dw.w, scores)
+        dsa.dsa_topk(scores, idx)
     dsa.dsa_sparse_mla_fwd(dw.q, dw.kv, idx, wl.scale, out, lse, p_sel, ws)
     res = {"scores": scores, "idx": idx, "out": out, "lse": lse, "p_sel": p_sel}
     if emit_p:

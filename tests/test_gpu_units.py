@@ -232,3 +232,38 @@ def test_kl_matches_oracle_rows_and_sum(dsa):
             total += e
     assert abs(loss.item() - total) <= parity.KL_RTOL * abs(total)
     assert loss.item() == loss2.item()
+
+
+# ----------------------------------------------------------------------------------- fused indexer -> top-k
+@pytest.mark.parametrize("H_I,B,Lk,k,w_den", [
+    (64, 5, 3000, 512, 16),      # 1-CTA rows, ragged tail tile
+    (64, 40, 20000, 2048, 16),   # 2-CTA clusters
+    (32, 7, 70000, 2048, 1),     # w in {-1, 0, 1}: heavy ties, 4-CTA clusters
+    (64, 3, 131072, 4096, 2),    # the longest rows and the largest k
+])
+def test_fused_indexer_topk_matches_the_two_calls_and_the_oracle(dsa, H_I, B, Lk, k, w_den):
+    wl = dsa_inputs.custom(f"fused_{H_I}_{Lk}", 2468 + Lk, B, 1, Lk, H_I, 128, w_den, k, 1, 16, 16)
+    dw = parity.DeviceWorkload(wl, with_attention=False)
+    s1 = torch.full((B, 1, Lk), float("nan"), device="cuda")
+    s2 = torch.full((B, 1, Lk), float("nan"), device="cuda")
+    i1 = torch.full((B, 1, k), -7, dtype=torch.int32, device="cuda")
+    i2 = torch.full((B, 1, k), -7, dtype=torch.int32, device="cuda")
+    ws = torch.full((dsa.dsa_workspace_bytes(dsa.DSA_OP_INDEXER_TOPK, B, 1, Lk, k, 0),), 0xAB,
+                    dtype=torch.uint8, device="cuda")  # garbage: the call clears what it uses
+    for _ in range(2):  # twice: the histograms start from zero on every call
+        dsa.dsa_indexer_topk(dw.qI, dw.kI, dw.w, s1, i1, ws)
+    dsa.dsa_indexer(dw.qI, dw.kI, dw.w, s2)
+    dsa.dsa_topk(s2, i2)
+    assert dsa.dsa_last_device_status() == 0
+    assert torch.equal(s1, s2) and torch.equal(i1, i2)
+    got = i1.cpu().numpy()
+    sc = s1.cpu().numpy()
+    for b in range(B):
+        exp, n = ref.topk_row(sc[b, 0].astype(np.float64), Lk - 1, k)
+        np.testing.assert_array_equal(got[b, 0], exp, err_msg=f"row {b}")
+    # the scores themselves are checked bit for bit on two rows
+    qI = dw.qI_np.reshape(B, H_I, 128)
+    w = dw.w_np.reshape(B, H_I)
+    for b in (0, B - 1):
+        exp = ref.indexer_row(qI[b], dw.kI_np[b], w[b], Lk - 1).astype(np.float32)
+        np.testing.assert_array_equal(sc[b, 0], exp)
