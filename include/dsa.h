@@ -192,6 +192,29 @@ dsa_status dsa_indexer_kl_dense(const float* scores, const float* p_full, int B,
                                 dsa_stream_t stream);
 
 /*
+ * Gradient of the indexer loss with respect to the indexer's inputs.  The indexer is trained
+ * from L^I alone, on a detached input ("DSA Continued Pre-Training" page, Stage 2; "DeepSeek-V3.2"
+ * analysis page, eq. (4) and the detached-input paragraph), so this is the whole training signal
+ * of q_I, w and k_I.  The selection is held fixed (top-k is piecewise constant); ReLU'(0) = 0:
+ *   g_i       = Softmax_i(scores[b,i,idx_i]) * sum_i p_i - p_i          (dL/dI over the slots)
+ *   dw[b,i,j] = sum_i g_i ReLU(a_ji),                a_ji = q_I[b,i,j,:] . k_I[b,idx_i,:]
+ *   dq[b,i,j,:] = sum_i g_i w[b,i,j] [a_ji > 0] k_I[b,idx_i,:]
+ *   dk[b,s,:] = sum over the queries i and slots with idx_i = s of g_i sum_j w[b,i,j] [a_ji > 0] q_I[b,i,j,:]
+ * Dense warm-up (eq. (3)): idx = NULL and k = Lk; every s <= t is a slot and p_sel is the
+ * [B, Lq, Lk] target of dsa_dense_mla_fwd.
+ *   q_fp8 [B,Lq,H_I,d_I] e4m3, k_fp8 [B,Lk,d_I] e4m3, w [B,Lq,H_I] fp32, scores [B,Lq,Lk] fp32
+ *   (dsa_indexer's output), idx [B,Lq,k] int32 (nullable), p_sel [B,Lq,k] fp32
+ *   dq [B,Lq,H_I,d_I] fp32, dw [B,Lq,H_I] fp32, dk [B,Lk,d_I] fp32 (all written; dk is cleared on
+ *   the stream, then accumulated with fp32 atomics, so its last bits depend on their order)
+ * The recomputed q_I . k_I products run on the FP8 tensor cores; the gradient products on the
+ * fp16 tensor cores with G split into two fp16 parts (inputs exact in fp16), fp32 accumulation.
+ * Supported: H_I = 64, d_I = 128, k <= 65536.
+ */
+dsa_status dsa_indexer_bwd(const void* q_fp8, const void* k_fp8, const float* w, const float* scores,
+                           const int32_t* idx, const float* p_sel, int B, int Lq, int Lk, int H_I,
+                           int d_I, int k, float* dq, float* dw, float* dk, dsa_stream_t stream);
+
+/*
  * The indexer loss of dsa_indexer_kl for callers that cannot hand the library any scratch
  * memory.  The pages have no counterpart to this entry point; it exists only for how memory
  * is provided.  Some callers cannot allocate device memory when they call in: a serving

@@ -19,7 +19,7 @@ __all__ = [
     "DsaError", "load", "dsa_status_str", "dsa_version", "dsa_workspace_bytes", "dsa_indexer",
     "dsa_topk", "dsa_sparse_mla_fwd", "dsa_indexer_kl", "dsa_indexer_kl_noalloc",
     "dsa_last_device_status", "dsa_set_wait_limit_ns", "dsa_selftest_wait", "dsa_dense_mla_fwd",
-    "dsa_indexer_kl_dense", "dsa_indexer_topk",
+    "dsa_indexer_kl_dense", "dsa_indexer_topk", "dsa_indexer_bwd",
     "DSA_OP_INDEXER", "DSA_OP_TOPK", "DSA_OP_SPARSE_MLA_FWD", "DSA_OP_INDEXER_KL",
     "DSA_OP_DENSE_MLA_FWD", "DSA_OP_INDEXER_KL_DENSE", "DSA_OP_INDEXER_TOPK", "EXPORTED",
 ]
@@ -29,7 +29,7 @@ DSA_OP_DENSE_MLA_FWD, DSA_OP_INDEXER_KL_DENSE, DSA_OP_INDEXER_TOPK = 4, 5, 6
 EXPORTED = ("dsa_status_str", "dsa_version", "dsa_workspace_bytes", "dsa_indexer", "dsa_topk",
             "dsa_sparse_mla_fwd", "dsa_indexer_kl", "dsa_indexer_kl_noalloc",
             "dsa_last_device_status", "dsa_set_wait_limit_ns", "dsa_selftest_wait",
-            "dsa_dense_mla_fwd", "dsa_indexer_kl_dense", "dsa_indexer_topk")
+            "dsa_dense_mla_fwd", "dsa_indexer_kl_dense", "dsa_indexer_topk", "dsa_indexer_bwd")
 
 
 class DsaError(RuntimeError):
@@ -67,9 +67,11 @@ def load(rebuild: bool = False) -> ctypes.CDLL:
         lib.dsa_dense_mla_fwd.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, f32, vp, vp, vp, vp, sz, vp]
         lib.dsa_indexer_kl_dense.argtypes = [vp, vp, i32, i32, i32, vp, vp, vp, sz, vp]
         lib.dsa_indexer_topk.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, sz, vp]
+        lib.dsa_indexer_bwd.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, vp, vp, vp]
         for name in ("dsa_indexer", "dsa_topk", "dsa_sparse_mla_fwd", "dsa_indexer_kl",
                      "dsa_indexer_kl_noalloc", "dsa_last_device_status", "dsa_set_wait_limit_ns",
-                     "dsa_selftest_wait", "dsa_dense_mla_fwd", "dsa_indexer_kl_dense", "dsa_indexer_topk"):
+                     "dsa_selftest_wait", "dsa_dense_mla_fwd", "dsa_indexer_kl_dense", "dsa_indexer_topk",
+                     "dsa_indexer_bwd"):
             getattr(lib, name).restype = i32
         _lib = lib
     return _lib
@@ -244,6 +246,29 @@ def dsa_indexer_kl_dense(scores: torch.Tensor, p_full: torch.Tensor, loss: torch
     _raise("dsa_indexer_kl_dense",
            load().dsa_indexer_kl_dense(_ptr(scores), _ptr(p_full), B, Lq, Lk, _ptr(loss),
                                        _ptr(loss_per_query), wsp, wsb, _stream(stream)))
+
+
+def dsa_indexer_bwd(q_fp8: torch.Tensor, k_fp8: torch.Tensor, w: torch.Tensor, scores: torch.Tensor,
+                    idx: torch.Tensor | None, p_sel: torch.Tensor, dq: torch.Tensor, dw: torch.Tensor,
+                    dk: torch.Tensor, stream=None) -> None:
+    """Gradients (dq, dw, dk) of the indexer loss with respect to q_I, w and k_I, the selection
+    idx held fixed (idx None: the dense warm-up loss over every s <= t, p_sel [B,Lq,Lk])."""
+    B, Lq, H_I, d_I = q_fp8.shape
+    Lk = k_fp8.shape[1]
+    k = Lk if idx is None else idx.shape[2]
+    _check(q_fp8, "q_fp8", torch.float8_e4m3fn, (B, Lq, H_I, d_I))
+    _check(k_fp8, "k_fp8", torch.float8_e4m3fn, (B, Lk, d_I))
+    _check(w, "w", torch.float32, (B, Lq, H_I))
+    _check(scores, "scores", torch.float32, (B, Lq, Lk))
+    if idx is not None:
+        _check(idx, "idx", torch.int32, (B, Lq, k))
+    _check(p_sel, "p_sel", torch.float32, (B, Lq, k))
+    _check(dq, "dq", torch.float32, (B, Lq, H_I, d_I))
+    _check(dw, "dw", torch.float32, (B, Lq, H_I))
+    _check(dk, "dk", torch.float32, (B, Lk, d_I))
+    _raise("dsa_indexer_bwd",
+           load().dsa_indexer_bwd(_ptr(q_fp8), _ptr(k_fp8), _ptr(w), _ptr(scores), _ptr(idx), _ptr(p_sel), B, Lq,
+                                  Lk, H_I, d_I, k, _ptr(dq), _ptr(dw), _ptr(dk), _stream(stream)))
 
 
 def dsa_indexer_kl_noalloc(scores: torch.Tensor, idx: torch.Tensor, p_sel: torch.Tensor,

@@ -13,6 +13,7 @@
 
 #include "../../include/dsa.h"
 #include "indexer.cuh"
+#include "indexer_bwd.cuh"
 #include "indexer_kl.cuh"
 #include "ptx.cuh"
 #include "sparse_mla.cuh"
@@ -631,6 +632,46 @@ dsa_status dsa_indexer_kl_dense(const float* scores, const float* p_full, int B,
   if (sr != DSA_OK) return sr;
   return launch(dsa::kl::kl_sum_kernel, 1u, dsa::kl::kSumThreads, 0, st, 1, static_cast<const float*>(per_row),
                 static_cast<int>(rows), loss);
+}
+
+dsa_status dsa_indexer_bwd(const void* q_fp8, const void* k_fp8, const float* w, const float* scores,
+                           const int32_t* idx, const float* p_sel, int B, int Lq, int Lk, int H_I, int d_I, int k,
+                           float* dq, float* dw, float* dk, dsa_stream_t stream) {
+  if (!q_fp8 || !k_fp8 || !w || !scores || !p_sel || !dq || !dw || !dk) return DSA_ERR_INVALID_ARG;
+  if (B <= 0 || Lq <= 0 || Lk <= 0 || Lq > Lk || H_I <= 0 || d_I <= 0 || k <= 0) return DSA_ERR_INVALID_ARG;
+  if (idx == nullptr && k != Lk) return DSA_ERR_INVALID_ARG;  // dense: every position is a slot
+  if (!aligned16(q_fp8) || !aligned16(k_fp8) || !aligned16(w) || !aligned16(scores) || (idx && !aligned16(idx)) ||
+      !aligned16(p_sel) || !aligned16(dq) || !aligned16(dw) || !aligned16(dk))
+    return DSA_ERR_INVALID_ARG;
+  if (H_I != dsa::bwd::kHI || d_I != dsa::bwd::kDI) return DSA_ERR_UNSUPPORTED;
+  if (static_cast<long>(B) * Lk >= INT32_MAX || static_cast<long>(B) * Lq >= INT32_MAX) return DSA_ERR_UNSUPPORTED;
+  DeviceInfo dev;
+  const dsa_status ds = current_device(dev);
+  if (ds != DSA_OK) return ds;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // dk accumulates over every query that selected a key
+  if (cudaMemsetAsync(dk, 0, static_cast<size_t>(B) * Lk * d_I * sizeof(float), st) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  dsa::bwd::Params p{};
+  p.q = static_cast<const uint8_t*>(q_fp8);
+  p.kI = static_cast<const uint8_t*>(k_fp8);
+  p.w = w;
+  p.scores = scores;
+  p.idx = idx;
+  p.p = p_sel;
+  p.dq = dq;
+  p.dw = dw;
+  p.dk = dk;
+  p.B = B;
+  p.Lq = Lq;
+  p.Lk = Lk;
+  p.k = k;
+  auto kern = dsa::bwd::indexer_bwd_kernel;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dsa::bwd::kSmemBytes) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  const long rows = static_cast<long>(B) * Lq;
+  const unsigned grid = static_cast<unsigned>(std::min<long>(rows, 2L * dev.sms));
+  return launch(kern, grid, dsa::bwd::kThreads, dsa::bwd::kSmemBytes, st, 1, p);
 }
 
 dsa_status dsa_set_wait_limit_ns(uint64_t ns) {
