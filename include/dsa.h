@@ -121,6 +121,41 @@ dsa_status dsa_indexer_topk(const void* q_fp8, const void* k_fp8, const float* w
                             size_t ws_bytes, dsa_stream_t stream);
 
 /*
+ * Decode over a paged cache with per-row lengths ("DeepSeek-V3.2" analysis page, sec. 5.1: a
+ * query's candidates may sit in a few contiguous cache pages or be spread over k pages, and a
+ * per-row seq_lens keeps a batch of different context lengths from being padded to the longest).
+ * The caches are pools of pages of page_size entries; sequence b's entry s sits in page
+ * block_table[b * max_pages + s / page_size] at row s % page_size, max_pages =
+ * ceil(max_len / page_size), and sequence b's query sees s < seq_lens[b] (t = seq_lens[b] - 1).
+ * Same results as dsa_indexer_topk / dsa_sparse_mla_fwd on each sequence's contiguous cache.
+ *   q_fp8 [B,1,H_I,d_I] e4m3, k_pages [num_pages,page_size,d_I] e4m3, w [B,1,H_I] fp32,
+ *   block_table [B, max_pages] int32, seq_lens [B] int32 (device; values outside [0, max_len]
+ *   are clamped and a page index outside [0, num_pages) reads as an empty entry, both recorded
+ *   as DSA_ERR_INVALID_ARG in the device status word)
+ *   scores [B,1,max_len] fp32 (-inf for s >= seq_lens[b]), idx [B,1,k] int32
+ *   ws: dsa_workspace_bytes(DSA_OP_INDEXER_TOPK, B, 1, max_len, k, 0) bytes
+ * Supported: (H_I, d_I) in {(64, 128), (32, 128)}, k <= 4096, max_len <= 262144.
+ */
+dsa_status dsa_indexer_topk_paged(const void* q_fp8, const void* k_pages, const float* w,
+                                  const int32_t* block_table, const int32_t* seq_lens, float* scores,
+                                  int32_t* idx, int B, int max_len, int num_pages, int page_size,
+                                  int H_I, int d_I, int k, void* ws, size_t ws_bytes,
+                                  dsa_stream_t stream);
+
+/*
+ * dsa_sparse_mla_fwd for decode over a paged latent cache (layout as dsa_indexer_topk_paged):
+ *   q_bf16 [B,1,H,576] bf16, kv_pages [num_pages,page_size,576] bf16, idx [B,1,k] int32
+ *   (positions within each sequence), out_bf16 [B,1,H,512], lse [B,1,H] (nullable)
+ *   ws: dsa_workspace_bytes(DSA_OP_SPARSE_MLA_FWD, B, 1, max_len, k, H) bytes
+ * Supported: (d_qk, d_v) = (576, 512), H <= 128, k <= 65536.
+ */
+dsa_status dsa_sparse_mla_fwd_paged(const void* q_bf16, const void* kv_pages, const int32_t* idx,
+                                    const int32_t* block_table, const int32_t* seq_lens, int B,
+                                    int max_len, int num_pages, int page_size, int H, int d_qk,
+                                    int d_v, int k, float scale, void* out_bf16, float* lse, void* ws,
+                                    size_t ws_bytes, dsa_stream_t stream);
+
+/*
  * Sparse attention in MLA's MQA mode over the selected latents ("DeepSeek-V3.2" analysis
  * page, sec. 1.1, eq. (2) and the MQA-mode paragraph; renormalised form eq. (19)).
  * Every query head shares the latent entry c_s = kv[b,s,:]; keys use all d_qk dims,

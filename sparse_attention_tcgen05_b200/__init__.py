@@ -19,7 +19,8 @@ __all__ = [
     "DsaError", "load", "dsa_status_str", "dsa_version", "dsa_workspace_bytes", "dsa_indexer",
     "dsa_topk", "dsa_sparse_mla_fwd", "dsa_indexer_kl", "dsa_indexer_kl_noalloc",
     "dsa_last_device_status", "dsa_set_wait_limit_ns", "dsa_selftest_wait", "dsa_dense_mla_fwd",
-    "dsa_indexer_kl_dense", "dsa_indexer_topk", "dsa_indexer_bwd",
+    "dsa_indexer_kl_dense", "dsa_indexer_topk", "dsa_indexer_bwd", "dsa_indexer_topk_paged",
+    "dsa_sparse_mla_fwd_paged",
     "DSA_OP_INDEXER", "DSA_OP_TOPK", "DSA_OP_SPARSE_MLA_FWD", "DSA_OP_INDEXER_KL",
     "DSA_OP_DENSE_MLA_FWD", "DSA_OP_INDEXER_KL_DENSE", "DSA_OP_INDEXER_TOPK", "EXPORTED",
 ]
@@ -29,7 +30,8 @@ DSA_OP_DENSE_MLA_FWD, DSA_OP_INDEXER_KL_DENSE, DSA_OP_INDEXER_TOPK = 4, 5, 6
 EXPORTED = ("dsa_status_str", "dsa_version", "dsa_workspace_bytes", "dsa_indexer", "dsa_topk",
             "dsa_sparse_mla_fwd", "dsa_indexer_kl", "dsa_indexer_kl_noalloc",
             "dsa_last_device_status", "dsa_set_wait_limit_ns", "dsa_selftest_wait",
-            "dsa_dense_mla_fwd", "dsa_indexer_kl_dense", "dsa_indexer_topk", "dsa_indexer_bwd")
+            "dsa_dense_mla_fwd", "dsa_indexer_kl_dense", "dsa_indexer_topk", "dsa_indexer_bwd",
+            "dsa_indexer_topk_paged", "dsa_sparse_mla_fwd_paged")
 
 
 class DsaError(RuntimeError):
@@ -68,10 +70,14 @@ def load(rebuild: bool = False) -> ctypes.CDLL:
         lib.dsa_indexer_kl_dense.argtypes = [vp, vp, i32, i32, i32, vp, vp, vp, sz, vp]
         lib.dsa_indexer_topk.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, sz, vp]
         lib.dsa_indexer_bwd.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, vp, vp, vp]
+        lib.dsa_indexer_topk_paged.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, vp,
+                                               sz, vp]
+        lib.dsa_sparse_mla_fwd_paged.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, f32,
+                                                 vp, vp, vp, sz, vp]
         for name in ("dsa_indexer", "dsa_topk", "dsa_sparse_mla_fwd", "dsa_indexer_kl",
                      "dsa_indexer_kl_noalloc", "dsa_last_device_status", "dsa_set_wait_limit_ns",
                      "dsa_selftest_wait", "dsa_dense_mla_fwd", "dsa_indexer_kl_dense", "dsa_indexer_topk",
-                     "dsa_indexer_bwd"):
+                     "dsa_indexer_bwd", "dsa_indexer_topk_paged", "dsa_sparse_mla_fwd_paged"):
             getattr(lib, name).restype = i32
         _lib = lib
     return _lib
@@ -269,6 +275,53 @@ def dsa_indexer_bwd(q_fp8: torch.Tensor, k_fp8: torch.Tensor, w: torch.Tensor, s
     _raise("dsa_indexer_bwd",
            load().dsa_indexer_bwd(_ptr(q_fp8), _ptr(k_fp8), _ptr(w), _ptr(scores), _ptr(idx), _ptr(p_sel), B, Lq,
                                   Lk, H_I, d_I, k, _ptr(dq), _ptr(dw), _ptr(dk), _stream(stream)))
+
+
+def dsa_indexer_topk_paged(q_fp8: torch.Tensor, k_pages: torch.Tensor, w: torch.Tensor,
+                           block_table: torch.Tensor, seq_lens: torch.Tensor, scores: torch.Tensor,
+                           idx: torch.Tensor, ws: torch.Tensor | None = None, stream=None) -> None:
+    """Decode indexer + top-k over a paged k_I cache: k_pages [num_pages, page_size, d_I] e4m3,
+    block_table [B, max_pages] int32, seq_lens [B] int32; scores [B,1,max_len], idx [B,1,k]."""
+    B, Lq, H_I, d_I = q_fp8.shape
+    num_pages, page_size = k_pages.shape[0], k_pages.shape[1]
+    max_len = scores.shape[2]
+    k = idx.shape[2]
+    _check(q_fp8, "q_fp8", torch.float8_e4m3fn, (B, 1, H_I, d_I))
+    _check(k_pages, "k_pages", torch.float8_e4m3fn, (num_pages, page_size, d_I))
+    _check(w, "w", torch.float32, (B, 1, H_I))
+    _check(block_table, "block_table", torch.int32, (B, -(-max_len // page_size)))
+    _check(seq_lens, "seq_lens", torch.int32, (B,))
+    _check(scores, "scores", torch.float32, (B, 1, max_len))
+    _check(idx, "idx", torch.int32, (B, 1, k))
+    wsp, wsb = _ws(ws)
+    _raise("dsa_indexer_topk_paged",
+           load().dsa_indexer_topk_paged(_ptr(q_fp8), _ptr(k_pages), _ptr(w), _ptr(block_table), _ptr(seq_lens),
+                                         _ptr(scores), _ptr(idx), B, max_len, num_pages, page_size, H_I, d_I, k,
+                                         wsp, wsb, _stream(stream)))
+
+
+def dsa_sparse_mla_fwd_paged(q: torch.Tensor, kv_pages: torch.Tensor, idx: torch.Tensor,
+                             block_table: torch.Tensor, seq_lens: torch.Tensor, max_len: int, scale: float,
+                             out: torch.Tensor, lse: torch.Tensor | None = None,
+                             ws: torch.Tensor | None = None, stream=None) -> None:
+    """Decode sparse MLA over a paged latent cache kv_pages [num_pages, page_size, 576] bf16."""
+    B, Lq, H, d_qk = q.shape
+    num_pages, page_size = kv_pages.shape[0], kv_pages.shape[1]
+    k = idx.shape[2]
+    d_v = out.shape[3]
+    _check(q, "q", torch.bfloat16, (B, 1, H, d_qk))
+    _check(kv_pages, "kv_pages", torch.bfloat16, (num_pages, page_size, d_qk))
+    _check(idx, "idx", torch.int32, (B, 1, k))
+    _check(block_table, "block_table", torch.int32, (B, -(-max_len // page_size)))
+    _check(seq_lens, "seq_lens", torch.int32, (B,))
+    _check(out, "out", torch.bfloat16, (B, 1, H, d_v))
+    if lse is not None:
+        _check(lse, "lse", torch.float32, (B, 1, H))
+    wsp, wsb = _ws(ws)
+    _raise("dsa_sparse_mla_fwd_paged",
+           load().dsa_sparse_mla_fwd_paged(_ptr(q), _ptr(kv_pages), _ptr(idx), _ptr(block_table), _ptr(seq_lens), B,
+                                           max_len, num_pages, page_size, H, d_qk, d_v, k, float(scale), _ptr(out),
+                                           _ptr(lse), wsp, wsb, _stream(stream)))
 
 
 def dsa_indexer_kl_noalloc(scores: torch.Tensor, idx: torch.Tensor, p_sel: torch.Tensor,

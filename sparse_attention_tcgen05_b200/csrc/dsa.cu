@@ -104,6 +104,15 @@ bool encode_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, ui
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// A paged decode cache: key/latent s of sequence b lives in row
+// block_table[b * max_pages + s / page_size] * page_size + s % page_size of the page pool, and
+// sequence b's context is seq_lens[b] long.
+struct Paging {
+  const int32_t* block_table;
+  const int32_t* seq_lens;
+  int page_size, max_pages, num_pages;
+};
+
 inline dsa_status launch_result() {
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
@@ -139,7 +148,8 @@ dsa_status launch(void (*kern)(KArgs...), unsigned grid, unsigned block, size_t 
 // ------------------------------------------------------------------------------ indexer
 template <int H_I, int D_I, int G>
 dsa_status launch_indexer(const void* q, const void* kk, const float* w, float* scores, int B,
-                          int Lq, int Lk, int sms, cudaStream_t stream, uint32_t* hist = nullptr) {
+                          int Lq, int Lk, int sms, cudaStream_t stream, uint32_t* hist = nullptr,
+                          const Paging* pg = nullptr) {
   using Cfg = dsa::indexer::Cfg<H_I, D_I, G>;
   const CUtensorMapSwizzle swz = D_I == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
                                  : D_I == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
@@ -148,11 +158,18 @@ dsa_status launch_indexer(const void* q, const void* kk, const float* w, float* 
   if (!encode_2d(&tm_q, CU_TENSOR_MAP_DATA_TYPE_UINT8, q, D_I, static_cast<uint64_t>(B) * Lq * H_I,
                  D_I, D_I, Cfg::N, swz))
     return DSA_ERR_CUDA;
-  if (!encode_2d(&tm_k, CU_TENSOR_MAP_DATA_TYPE_UINT8, kk, D_I, static_cast<uint64_t>(B) * Lk, D_I,
-                 D_I, dsa::indexer::kTileKeys, swz))
+  const uint64_t k_rows = pg ? static_cast<uint64_t>(pg->num_pages) * pg->page_size : static_cast<uint64_t>(B) * Lk;
+  if (!encode_2d(&tm_k, CU_TENSOR_MAP_DATA_TYPE_UINT8, kk, D_I, k_rows, D_I, D_I, dsa::indexer::kTileKeys, swz))
     return DSA_ERR_CUDA;
   dsa::indexer::Params p{};
   p.k = static_cast<const uint8_t*>(kk);
+  if (pg) {
+    p.block_table = pg->block_table;
+    p.seq_lens = pg->seq_lens;
+    p.page_size = pg->page_size;
+    p.max_pages = pg->max_pages;
+    p.num_pages = pg->num_pages;
+  }
   p.w = w;
   p.scores = scores;
   p.hist = hist;
@@ -185,13 +202,13 @@ dsa_status launch_indexer(const void* q, const void* kk, const float* w, float* 
 // ------------------------------------------------------------------------------ top-k
 template <int C, int KPT>
 dsa_status launch_topk(const float* scores, int32_t* idx, int B, int Lq, int Lk, int k,
-                       cudaStream_t stream, const uint32_t* ghist) {
+                       cudaStream_t stream, const uint32_t* ghist, const int32_t* seq_lens) {
   auto kern = dsa::topk::topk_kernel<C, KPT>;
   constexpr int smem = dsa::topk::dyn_smem_bytes<KPT>();
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return DSA_ERR_CUDA;
   return launch(kern, static_cast<unsigned>(B) * Lq * C, dsa::topk::kThreads, smem, stream, C, scores, idx, B, Lq,
-                Lk, k, ghist);
+                Lk, k, ghist, seq_lens);
 }
 
 // Keys per CTA for a row split over c CTAs (a multiple of 4, as the kernel computes it).
@@ -207,35 +224,37 @@ int topk_cluster_size(int rows, int Lk, int sms) {
 
 template <int C>
 dsa_status launch_topk_c(const float* scores, int32_t* idx, int B, int Lq, int Lk, int k,
-                         cudaStream_t st, const uint32_t* ghist) {
+                         cudaStream_t st, const uint32_t* ghist, const int32_t* sl) {
   const int slice = topk_slice(Lk, C);
-  if (slice <= 4 * dsa::topk::kThreads) return launch_topk<C, 4>(scores, idx, B, Lq, Lk, k, st, ghist);
-  if (slice <= 8 * dsa::topk::kThreads) return launch_topk<C, 8>(scores, idx, B, Lq, Lk, k, st, ghist);
-  if (slice <= 16 * dsa::topk::kThreads) return launch_topk<C, 16>(scores, idx, B, Lq, Lk, k, st, ghist);
-  return launch_topk<C, 32>(scores, idx, B, Lq, Lk, k, st, ghist);
+  if (slice <= 4 * dsa::topk::kThreads) return launch_topk<C, 4>(scores, idx, B, Lq, Lk, k, st, ghist, sl);
+  if (slice <= 8 * dsa::topk::kThreads) return launch_topk<C, 8>(scores, idx, B, Lq, Lk, k, st, ghist, sl);
+  if (slice <= 16 * dsa::topk::kThreads) return launch_topk<C, 16>(scores, idx, B, Lq, Lk, k, st, ghist, sl);
+  return launch_topk<C, 32>(scores, idx, B, Lq, Lk, k, st, ghist, sl);
 }
 
-// Top-k with the validated sizes; ghist (nullable) holds each row's top-digit counts.
+// Top-k with the validated sizes; ghist (nullable) holds each row's top-digit counts, seq_lens
+// (nullable, Lq == 1) each row's context length.
 dsa_status run_topk(const float* scores, int32_t* idx, int B, int Lq, int Lk, int k, int sms, cudaStream_t st,
-                    const uint32_t* ghist) {
+                    const uint32_t* ghist, const int32_t* seq_lens = nullptr) {
   switch (topk_cluster_size(B * Lq, Lk, sms)) {
-    case 1: return launch_topk_c<1>(scores, idx, B, Lq, Lk, k, st, ghist);
-    case 2: return launch_topk_c<2>(scores, idx, B, Lq, Lk, k, st, ghist);
-    case 4: return launch_topk_c<4>(scores, idx, B, Lq, Lk, k, st, ghist);
-    default: return launch_topk_c<8>(scores, idx, B, Lq, Lk, k, st, ghist);
+    case 1: return launch_topk_c<1>(scores, idx, B, Lq, Lk, k, st, ghist, seq_lens);
+    case 2: return launch_topk_c<2>(scores, idx, B, Lq, Lk, k, st, ghist, seq_lens);
+    case 4: return launch_topk_c<4>(scores, idx, B, Lq, Lk, k, st, ghist, seq_lens);
+    default: return launch_topk_c<8>(scores, idx, B, Lq, Lk, k, st, ghist, seq_lens);
   }
 }
 
 // Indexer with the validated sizes.  hist (nullable, decode kernels only) receives each row's
 // top-digit counts; returns DSA_ERR_UNSUPPORTED for shapes outside the compiled kernels.
 dsa_status run_indexer(const void* q_fp8, const void* k_fp8, const float* w, float* scores, int B, int Lq, int Lk,
-                       int H_I, int d_I, int sms, cudaStream_t st, uint32_t* hist) {
+                       int H_I, int d_I, int sms, cudaStream_t st, uint32_t* hist, const Paging* pg = nullptr) {
   const bool decode = (Lq == 1);
+  if (pg && !(decode && d_I == 128 && (H_I == 64 || H_I == 32))) return DSA_ERR_UNSUPPORTED;
   if (H_I == 64 && d_I == 128)
-    return decode ? launch_indexer<64, 128, 1>(q_fp8, k_fp8, w, scores, B, Lq, Lk, sms, st, hist)
+    return decode ? launch_indexer<64, 128, 1>(q_fp8, k_fp8, w, scores, B, Lq, Lk, sms, st, hist, pg)
                   : launch_indexer<64, 128, 4>(q_fp8, k_fp8, w, scores, B, Lq, Lk, sms, st);
   if (H_I == 32 && d_I == 128)
-    return decode ? launch_indexer<32, 128, 1>(q_fp8, k_fp8, w, scores, B, Lq, Lk, sms, st, hist)
+    return decode ? launch_indexer<32, 128, 1>(q_fp8, k_fp8, w, scores, B, Lq, Lk, sms, st, hist, pg)
                   : launch_indexer<32, 128, 8>(q_fp8, k_fp8, w, scores, B, Lq, Lk, sms, st);
   if (H_I == 16 && d_I == 128) return launch_indexer<16, 128, 16>(q_fp8, k_fp8, w, scores, B, Lq, Lk, sms, st);
   if (H_I == 8 && d_I == 64) return launch_indexer<8, 64, 32>(q_fp8, k_fp8, w, scores, B, Lq, Lk, sms, st);
@@ -277,7 +296,8 @@ size_t mla_ws_bytes(int rows, int k, int H, int d_v, int sms) {
 template <int D_QK, int D_V>
 dsa_status launch_mla(const void* q, const void* kv, const int32_t* idx, int B, int Lq, int Lk,
                       int H, int k, float scale, void* out, float* lse, float* p_sel, void* ws,
-                      size_t ws_bytes, int sms, cudaStream_t stream, int dense = 0) {
+                      size_t ws_bytes, int sms, cudaStream_t stream, int dense = 0,
+                      const Paging* pg = nullptr) {
   using Cfg = dsa::mla::Cfg<D_QK, D_V>;
   const int rows = B * Lq;
   const MlaSplit sp = mla_split(rows, k, Cfg::kNdv, sms, p_sel != nullptr);
@@ -297,6 +317,16 @@ dsa_status launch_mla(const void* q, const void* kv, const int32_t* idx, int B, 
   p.per_split = sp.per_split;
   p.scale_log2 = scale * dsa::mla::kLog2e;
   p.dense = dense;
+  const long kv_rows = pg ? static_cast<long>(pg->num_pages) * pg->page_size : static_cast<long>(B) * Lk;
+  if (kv_rows >= INT32_MAX) return DSA_ERR_UNSUPPORTED;
+  p.kv_rows = static_cast<int>(kv_rows);
+  if (pg) {
+    p.block_table = pg->block_table;
+    p.seq_lens = pg->seq_lens;
+    p.page_size = pg->page_size;
+    p.max_pages = pg->max_pages;
+    p.num_pages = pg->num_pages;
+  }
   if (sp.n_split > 1) {
     const size_t need = static_cast<size_t>(sp.n_split) * rows * H * (static_cast<size_t>(D_V) + 1) * sizeof(float);
     if (ws == nullptr || ws_bytes < need || !aligned16(ws)) return DSA_ERR_INVALID_ARG;
@@ -312,9 +342,9 @@ dsa_status launch_mla(const void* q, const void* kv, const int32_t* idx, int B, 
     // kv as [B * Lk rows, 576 dims]: one-row boxes of 64 dims (SW128) and of the 32 rope dims
     // (SW64) for the row gathers
     CUtensorMap tm_main, tm_rope;
-    if (!encode_2d(&tm_main, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kv, D_QK, static_cast<uint64_t>(B) * Lk,
+    if (!encode_2d(&tm_main, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kv, D_QK, static_cast<uint64_t>(kv_rows),
                    static_cast<uint64_t>(D_QK) * 2, 64, 1, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !encode_2d(&tm_rope, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kv, D_QK, static_cast<uint64_t>(B) * Lk,
+        !encode_2d(&tm_rope, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kv, D_QK, static_cast<uint64_t>(kv_rows),
                    static_cast<uint64_t>(D_QK) * 2, 32, 1, CU_TENSOR_MAP_SWIZZLE_64B))
       return DSA_ERR_CUDA;
     // q as [rows * H, 576]: 128 head rows x 64 dims (SW128) and x the 32 rope dims (SW64)
@@ -672,6 +702,66 @@ dsa_status dsa_indexer_bwd(const void* q_fp8, const void* k_fp8, const float* w,
   const long rows = static_cast<long>(B) * Lq;
   const unsigned grid = static_cast<unsigned>(std::min<long>(rows, 2L * dev.sms));
   return launch(kern, grid, dsa::bwd::kThreads, dsa::bwd::kSmemBytes, st, 1, p);
+}
+
+// Shared checks of the paged decode entry points; fills *pg.
+dsa_status check_paging(const int32_t* block_table, const int32_t* seq_lens, int B, int max_len, int num_pages,
+                        int page_size, Paging* pg) {
+  if (!block_table || !seq_lens) return DSA_ERR_INVALID_ARG;
+  if (B <= 0 || max_len <= 0 || num_pages <= 0 || page_size <= 0) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(block_table) || !aligned16(seq_lens)) return DSA_ERR_INVALID_ARG;
+  if (static_cast<long>(num_pages) * page_size >= INT32_MAX || static_cast<long>(B) * max_len >= INT32_MAX)
+    return DSA_ERR_UNSUPPORTED;
+  pg->block_table = block_table;
+  pg->seq_lens = seq_lens;
+  pg->page_size = page_size;
+  pg->max_pages = (max_len + page_size - 1) / page_size;
+  pg->num_pages = num_pages;
+  return DSA_OK;
+}
+
+dsa_status dsa_indexer_topk_paged(const void* q_fp8, const void* k_pages, const float* w, const int32_t* block_table,
+                                  const int32_t* seq_lens, float* scores, int32_t* idx, int B, int max_len,
+                                  int num_pages, int page_size, int H_I, int d_I, int k, void* ws, size_t ws_bytes,
+                                  dsa_stream_t stream) {
+  if (!q_fp8 || !k_pages || !w || !scores || !idx || H_I <= 0 || d_I <= 0 || k <= 0) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q_fp8) || !aligned16(k_pages) || !aligned16(w) || !aligned16(scores) || !aligned16(idx))
+    return DSA_ERR_INVALID_ARG;
+  Paging pg;
+  const dsa_status sp = check_paging(block_table, seq_lens, B, max_len, num_pages, page_size, &pg);
+  if (sp != DSA_OK) return sp;
+  if (!fused_topk_shape(1, H_I, d_I)) return DSA_ERR_UNSUPPORTED;
+  if (k > 4096 || topk_slice(max_len, 8) > dsa::topk::kMaxSlice) return DSA_ERR_UNSUPPORTED;
+  const size_t need = static_cast<size_t>(B) * 2048 * sizeof(uint32_t);
+  if (ws == nullptr || ws_bytes < need || !aligned16(ws)) return DSA_ERR_INVALID_ARG;
+  DeviceInfo dev;
+  const dsa_status ds = current_device(dev);
+  if (ds != DSA_OK) return ds;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t* hist = static_cast<uint32_t*>(ws);
+  if (cudaMemsetAsync(hist, 0, need, st) != cudaSuccess) return DSA_ERR_CUDA;
+  const dsa_status si = run_indexer(q_fp8, k_pages, w, scores, B, 1, max_len, H_I, d_I, dev.sms, st, hist, &pg);
+  if (si != DSA_OK) return si;
+  return run_topk(scores, idx, B, 1, max_len, k, dev.sms, st, hist, seq_lens);
+}
+
+dsa_status dsa_sparse_mla_fwd_paged(const void* q_bf16, const void* kv_pages, const int32_t* idx,
+                                    const int32_t* block_table, const int32_t* seq_lens, int B, int max_len,
+                                    int num_pages, int page_size, int H, int d_qk, int d_v, int k, float scale,
+                                    void* out_bf16, float* lse, void* ws, size_t ws_bytes, dsa_stream_t stream) {
+  if (!q_bf16 || !kv_pages || !idx || !out_bf16 || H <= 0 || k <= 0) return DSA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q_bf16) || !aligned16(kv_pages) || !aligned16(idx) || !aligned16(out_bf16) || (lse && !aligned16(lse)))
+    return DSA_ERR_INVALID_ARG;
+  Paging pg;
+  const dsa_status sp = check_paging(block_table, seq_lens, B, max_len, num_pages, page_size, &pg);
+  if (sp != DSA_OK) return sp;
+  if (d_qk != 576 || d_v != 512 || H > 128 || k > 65536) return DSA_ERR_UNSUPPORTED;
+  DeviceInfo dev;
+  const dsa_status ds = current_device(dev);
+  if (ds != DSA_OK) return ds;
+  return launch_mla<576, 512>(q_bf16, kv_pages, idx, B, 1, max_len, H, k, scale, out_bf16, lse, nullptr, ws, ws_bytes,
+                              dev.sms, static_cast<cudaStream_t>(stream), 0, &pg);
 }
 
 dsa_status dsa_set_wait_limit_ns(uint64_t ns) {

@@ -40,6 +40,12 @@ struct Params {
   const float* w;
   float* scores;
   uint32_t* hist;    // nullable, decode only: [B * Lq][2048] counts of the scores' top digit
+  // Paged decode cache (nullable block_table): key s of sequence b is row
+  // block_table[b * max_pages + s / page_size] * page_size + s % page_size of k, and the query
+  // sits at t = seq_lens[b] - 1 (clamped to [-1, Lk - 1]; Lk is then the longest context).
+  const int32_t* block_table;
+  const int32_t* seq_lens;
+  int page_size, max_pages, num_pages;
   int B, Lq, Lk;
   int n_qg;   // query groups per sequence
   int n_kt;   // key tiles per sequence
@@ -94,16 +100,35 @@ __device__ __forceinline__ void decode_item(const Params& p, int u, int& b, int&
   qg = p.n_qg - 1 - qg_rev;
 }
 
+// Position of query i of sequence b: i + Lk - Lq, or seq_lens[b] - 1 for a paged decode cache.
+__device__ __forceinline__ int query_pos(const Params& p, int b, int i) {
+  if (p.seq_lens == nullptr) return i + p.Lk - p.Lq;
+  const int n = __ldg(p.seq_lens + b);
+  if (n > p.Lk) record_bad_index();
+  return min(max(n, 0), p.Lk) - 1;
+}
+
 // Tiles [kt0, kt1) of the item; the first n_comp of them hold visible keys and need the MMA.
 template <int G>
-__device__ __forceinline__ void item_tiles(const Params& p, int qg, int kc, int& kt0, int& kt1,
+__device__ __forceinline__ void item_tiles(const Params& p, int b, int qg, int kc, int& kt0, int& kt1,
                                            int& n_comp) {
   kt0 = kc * p.kc;
   kt1 = min(kt0 + p.kc, p.n_kt);
   const int i_last = min(qg * G + G, p.Lq) - 1;
-  const int t_max = i_last + (p.Lk - p.Lq);
-  const int last_visible_tile = t_max / kTileKeys;
+  const int t_max = query_pos(p, b, i_last);
+  const int last_visible_tile = t_max < 0 ? -1 : t_max / kTileKeys;
   n_comp = max(0, min(kt1, last_visible_tile + 1) - kt0);
+}
+
+// Row of k holding key s of sequence b (-1: no such key).
+__device__ __forceinline__ long key_row(const Params& p, int b, int s) {
+  if (p.block_table == nullptr) return static_cast<long>(b) * p.Lk + s;
+  const int page = __ldg(p.block_table + static_cast<size_t>(b) * p.max_pages + s / p.page_size);
+  if (static_cast<unsigned>(page) >= static_cast<unsigned>(p.num_pages)) {
+    record_bad_index();
+    return -1;
+  }
+  return static_cast<long>(page) * p.page_size + s % p.page_size;
 }
 
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
@@ -168,7 +193,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int u = blockIdx.x; u < p.n_items; u += gridDim.x) {
         int b, qg, kc, kt0, kt1, n_comp;
         decode_item(p, u, b, qg, kc);
-        item_tiles<G>(p, qg, kc, kt0, kt1, n_comp);
+        item_tiles<G>(p, b, qg, kc, kt0, kt1, n_comp);
         if (n_comp == 0) continue;
         const int qb = qi & 1;
         const uint32_t qph = (qi >> 1) & 1;
@@ -189,7 +214,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // waits for tile j to be consumed, which needs only tiles <= j signalled (lag < stages) and
     // the q_I group of tile j's item, loaded by warp 3 once the item two back is consumed.
     const int pt = (warp == 0 ? 0 : 32) + lane;
-    const size_t k_rows = static_cast<size_t>(p.B) * p.Lk;
+    const size_t k_rows = p.block_table ? static_cast<size_t>(p.num_pages) * p.page_size
+                                        : static_cast<size_t>(p.B) * p.Lk;
     // k_I is read once: its lines go first out of L2, so that the scores written meanwhile stay
     // there for the top-k that reads them next
     const uint64_t evict_first = l2_evict_first_policy();
@@ -200,19 +226,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int u = blockIdx.x; ok && u < p.n_items; u += gridDim.x) {
       int b, qg, kc, kt0, kt1, n_comp;
       decode_item(p, u, b, qg, kc);
-      item_tiles<G>(p, qg, kc, kt0, kt1, n_comp);
+      item_tiles<G>(p, b, qg, kc, kt0, kt1, n_comp);
       for (int tt = 0; tt < n_comp; ++tt) {
         if (!mbar_wait(&k_empty[ks], kph ^ 1, abort_flag, 2)) {
           ok = false;
           break;
         }
-        const size_t row0 = static_cast<size_t>(b) * p.Lk + static_cast<size_t>(kt0 + tt) * kTileKeys;
+        const int s0 = (kt0 + tt) * kTileKeys;
         const uint32_t dst = smem_u32(sK + ks * C::kKBytes);
         for (int c = pt; c < kTileKeys * (D_I / 16); c += kLoadThreads) {
           const int r = c >> 3, ch = c & 7;
-          const bool valid = row0 + r < k_rows;  // rows past the tensor are zero-filled
-          cp_async_16_hint(dst + swizzled_offset(r, ch, 128), p.k + (valid ? (row0 + r) * D_I + ch * 16 : 0), valid,
-                           evict_first);
+          // keys past the sequence (or past the tensor) are zero-filled
+          const long kr = s0 + r < p.Lk ? key_row(p, b, s0 + r) : -1;
+          const bool valid = kr >= 0 && static_cast<size_t>(kr) < k_rows;
+          cp_async_16_hint(dst + swizzled_offset(r, ch, 128), p.k + (valid ? static_cast<size_t>(kr) * D_I + ch * 16 : 0),
+                           valid, evict_first);
         }
         cp_async_commit();
         if (++pending > kLoadLag) {
@@ -246,7 +274,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int u = blockIdx.x; u < p.n_items; u += gridDim.x) {
         int b, qg, kc, kt0, kt1, n_comp;
         decode_item(p, u, b, qg, kc);
-        item_tiles<G>(p, qg, kc, kt0, kt1, n_comp);
+        item_tiles<G>(p, b, qg, kc, kt0, kt1, n_comp);
         if (n_comp == 0) continue;
         const int qb = qi & 1;
         const uint32_t qph = (qi >> 1) & 1;
@@ -278,7 +306,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int u = blockIdx.x; u < p.n_items; u += gridDim.x) {
         int b, qg, kc, kt0, kt1, n_comp;
         decode_item(p, u, b, qg, kc);
-        item_tiles<G>(p, qg, kc, kt0, kt1, n_comp);
+        item_tiles<G>(p, b, qg, kc, kt0, kt1, n_comp);
         if (n_comp == 0) continue;
         const int qb = qi & 1;
         const uint32_t qph = (qi >> 1) & 1;
@@ -326,7 +354,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int u = blockIdx.x; u < p.n_items; u += gridDim.x, ++it) {
       int b, qg, kc, kt0, kt1, n_comp;
       decode_item(p, u, b, qg, kc);
-      item_tiles<G>(p, qg, kc, kt0, kt1, n_comp);
+      item_tiles<G>(p, b, qg, kc, kt0, kt1, n_comp);
       const int i0 = qg * G;
       float* wbuf = sW + (it & 1) * C::N;
       for (int x = e; x < C::N; x += 256) {
@@ -369,7 +397,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int g = 0; g < C::kQPerWG; ++g) {
             const int i = i0 + wg * C::kQPerWG * (C::kSplitWG ? 1 : 0) + g;
             if (i < p.Lq) {
-              const int t = i + p.Lk - p.Lq;
+              const int t = query_pos(p, b, i);
               p.scores[(row_base + i) * p.Lk + s] = (s <= t) ? acc[g] : -INFINITY;
               if (G == 1 && count && s <= t) atomicAdd(&sHist[ordered_key(acc[g]) >> 21], 1u);
             }

@@ -51,7 +51,32 @@ struct Params {
                            // cluster of four and combine in the kernel (no combine launch)
   int dense;               // dense causal attention: no idx, slot j is position j for j <= t,
                            // k == Lk (the dense warm-up's main attention and its target p)
+  // Paged decode cache (576-d kernel; nullable block_table): latent s of sequence b is row
+  // block_table[b * max_pages + s / page_size] * page_size + s % page_size of kv, and only
+  // s < seq_lens[b] are valid.  kv_rows: rows of the kv tensor (one past is the zero-fill row).
+  const int32_t* block_table;
+  const int32_t* seq_lens;
+  int page_size, max_pages, num_pages;
+  int kv_rows;
 };
+
+// Valid latent positions of sequence b: [0, Lk), or [0, seq_lens[b]) for a paged cache.
+__device__ __forceinline__ int row_len(const Params& p, int b) {
+  return p.seq_lens ? min(max(__ldg(p.seq_lens + b), 0), p.Lk) : p.Lk;
+}
+
+// Row of kv holding latent s of sequence b; kv_rows (one past the tensor, zero-filled by the
+// TMA) for an empty slot.
+__device__ __forceinline__ int kv_row(const Params& p, int b, int len_b, int s) {
+  if (static_cast<unsigned>(s) >= static_cast<unsigned>(len_b)) return p.kv_rows;
+  if (p.block_table == nullptr) return b * p.Lk + s;
+  const int page = __ldg(p.block_table + static_cast<size_t>(b) * p.max_pages + s / p.page_size);
+  if (static_cast<unsigned>(page) >= static_cast<unsigned>(p.num_pages)) {
+    record_bad_index();
+    return p.kv_rows;
+  }
+  return page * p.page_size + s % p.page_size;
+}
 
 // Query row served by the r-th row of the grid: in dense mode the latest (longest) rows go
 // first, so that the shortest ones fill the tail.

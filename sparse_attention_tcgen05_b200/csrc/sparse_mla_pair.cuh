@@ -290,8 +290,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // which needs pair jp landed.  Lane r holds the r-th index of each block of the pair;
     // invalid slots (and the missing half of an odd last pair) point one row past the tensor,
     // which the TMA fills with zeros.
-    const int row0 = b * p.Lk;
-    const int oob = p.B * p.Lk;
+    const int len_b = mla::row_len(p, b);
     const int w = warp - kGatherWarp0;
     const int op = w + kGatherWarps * lane;  // this lane's operation of each stage
     const bool has_op = lane < 12 && op < 80;
@@ -319,9 +318,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         next_lo = slot_of(2 * jp + 2);
         next_hi = slot_of(2 * jp + 3);
       }
-      if (s_lo >= p.Lk || s_hi >= p.Lk) record_bad_index();
-      const int y_lo = (static_cast<unsigned>(s_lo) < static_cast<unsigned>(p.Lk)) ? row0 + s_lo : oob;
-      const int y_hi = (static_cast<unsigned>(s_hi) < static_cast<unsigned>(p.Lk)) ? row0 + s_hi : oob;
+      if (s_lo >= len_b || s_hi >= len_b) record_bad_index();
+      const int y_lo = mla::kv_row(p, b, len_b, s_lo);
+      const int y_hi = mla::kv_row(p, b, len_b, s_hi);
       const int src = 4 * (g & 7);
       int yv[4];
 #pragma unroll
@@ -398,8 +397,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     auto blk_of = [&](int q) { return q < nblk ? q : q - nblk; };
+    const int len_s = mla::row_len(p, b);
     auto mask_of = [&](int s) {
-      return __ballot_sync(0xFFFFFFFFu, static_cast<unsigned>(s) < static_cast<unsigned>(p.Lk));
+      return __ballot_sync(0xFFFFFFFFu, static_cast<unsigned>(s) < static_cast<unsigned>(len_s));
     };
 
     // Steps 1-2 for block q: z[] = the full S(q) (unscaled), -inf at invalid slots.

@@ -205,7 +205,7 @@ __device__ __forceinline__ uint2 block_exclusive2(uint32_t a, uint32_t b, uint32
 template <int C, int KPT>
 __global__ void __launch_bounds__(kThreads, 1)
     topk_kernel(const float* __restrict__ scores, int32_t* __restrict__ idx, int B, int Lq, int Lk,
-                int k, const uint32_t* __restrict__ ghist) {
+                int k, const uint32_t* __restrict__ ghist, const int32_t* __restrict__ seq_lens) {
   static_assert(KPT == 4 || KPT == 8 || KPT == 16 || KPT == 32, "keys per thread");
   static_assert(C == 1 || C == 2 || C == 4 || C == kMaxCluster, "cluster size");
   constexpr int kCpr = KPT / 4;  // chunks per thread
@@ -226,7 +226,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int row = blockIdx.x / C;
   const uint32_t rank = (C > 1) ? cluster_ctarank() : 0u;
   const int i = row % Lq;
-  const int t = i + Lk - Lq;
+  // decode rows of a paged cache (Lq == 1) see their own context length, clamped to [0, Lk]
+  const int t = seq_lens ? min(max(__ldg(seq_lens + row / Lq), 0), Lk) - 1 : i + Lk - Lq;
   const int n = t + 1;  // candidates s in [0, n)
   int32_t* out = idx + static_cast<size_t>(row) * k;
   const int tid = threadIdx.x;
