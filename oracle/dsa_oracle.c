@@ -19,6 +19,9 @@
  *   - dense warm-up loss L^I = sum_t KL(p[t,:] || Softmax(I[t,:])) over every s <= t, with p
  *     the dense main attention summed over heads and L1-normalised, "DSA Continued
  *     Pre-Training" page, Stage 1, and the analysis page eq. (3)
+ *   - HISA's two-stage retrieval: blocks scored by a block representative, the best blocks'
+ *     tokens scored exactly, top-k among them (analysis page, sec. 5.3, eq. (24)-(25) and the
+ *     block-mean paragraph)
  *   - the gradient of one row's L^I with respect to the indexer's inputs q_I, w and k_I (the
  *     indexer is trained from L^I alone, on a detached input: "DSA Continued Pre-Training",
  *     Stage 2), with the selected set held fixed (top-k is piecewise constant)
@@ -244,6 +247,93 @@ double ref_dense_kl_row(const double* scores_row, int t, const double* p) {
     kl += p[s] * (log(p[s]) - (scores_row[s] - log_z));
   }
   return kl;
+}
+
+/* ---- f4: HISA, block -> token retrieval (analysis page, sec. 5.3) ----------------------- */
+/* Representative of a block of keys: the mean of its keys [s0, s0 + n) (the block-mean
+ * representation the page discusses).  k_seq: [..][d_I] e4m3; mean: [d_I]. */
+void ref_block_mean(const uint8_t* k_seq, int s0, int n, int d_I, double* mean) {
+  for (int d = 0; d < d_I; ++d) {
+    double acc = 0.0;
+    for (int s = s0; s < s0 + n; ++s) acc += ref_e4m3_to_double(k_seq[(int64_t)s * d_I + d]);
+    mean[d] = acc / (double)n;
+  }
+}
+
+/* Coarse score of a block for one query: the indexer's score formula with the block's mean
+ * key in place of a token key, sum_j w_j ReLU(q_j . mean). */
+double ref_block_score(const uint8_t* q_row, const double* mean, const float* w_row, int H_I, int d_I) {
+  double score = 0.0;
+  for (int j = 0; j < H_I; ++j) {
+    double dot = 0.0;
+    for (int d = 0; d < d_I; ++d) dot += ref_e4m3_to_double(q_row[j * d_I + d]) * mean[d];
+    score += (double)w_row[j] * (dot > 0.0 ? dot : 0.0);
+  }
+  return score;
+}
+
+/* HISA selection for query t: the keys are cut into blocks [b*bsize, b*bsize + bsize); a block
+ * starting at or before t is a candidate, represented by the mean of its keys s <= t; the r
+ * candidate blocks with the largest coarse scores are kept (ties -> smaller block); their keys
+ * s <= t form U; every key of U gets its exact indexer score (eq. (1)); S = the min(k, |U|) keys
+ * of U with the largest scores (ties -> smaller position).
+ * idx [k]: S ascending, -1 padded.  blocks [r]: the kept blocks ascending, -1 padded.
+ * Returns |S|. */
+int ref_hisa_row(const uint8_t* q_row, const uint8_t* k_seq, const float* w_row, int Lk, int t, int H_I,
+                 int d_I, int bsize, int r, int k, int32_t* idx, int32_t* blocks) {
+  int nb = t / bsize + 1; /* candidate blocks: those starting at or before t */
+  double* bscore = (double*)malloc(sizeof(double) * (size_t)nb);
+  double* mean = (double*)malloc(sizeof(double) * (size_t)d_I);
+  for (int b = 0; b < nb; ++b) {
+    int s0 = b * bsize;
+    int n = (t + 1 - s0) < bsize ? (t + 1 - s0) : bsize;
+    ref_block_mean(k_seq, s0, n, d_I, mean);
+    bscore[b] = ref_block_score(q_row, mean, w_row, H_I, d_I);
+  }
+  /* the r best blocks: the same full sort and tie rule as the token top-k */
+  int32_t* bsel = (int32_t*)malloc(sizeof(int32_t) * (size_t)(r > 0 ? r : 1));
+  int nsel = ref_topk_row(bscore, nb - 1, r, bsel);
+  for (int i = 0; i < r; ++i) blocks[i] = bsel[i];
+  /* exact scores on U (every other key -inf), then the token top-k */
+  double* sc = (double*)malloc(sizeof(double) * (size_t)(t + 1));
+  for (int s = 0; s <= t; ++s) sc[s] = -INFINITY;
+  int n_u = 0;
+  double* one = (double*)malloc(sizeof(double) * (size_t)Lk);
+  ref_indexer_row(q_row, k_seq, w_row, Lk, t, H_I, d_I, one);
+  for (int i = 0; i < nsel; ++i) {
+    int s0 = bsel[i] * bsize;
+    for (int s = s0; s < s0 + bsize && s <= t; ++s) {
+      sc[s] = one[s];
+      ++n_u;
+    }
+  }
+  /* top-k over U: rank the keys of U only (the others are not candidates) */
+  scored_t* c = (scored_t*)malloc(sizeof(scored_t) * (size_t)(n_u > 0 ? n_u : 1));
+  int m = 0;
+  for (int i = 0; i < nsel; ++i) {
+    int s0 = bsel[i] * bsize;
+    for (int s = s0; s < s0 + bsize && s <= t; ++s) {
+      c[m].score = sc[s];
+      c[m].s = s;
+      ++m;
+    }
+  }
+  qsort(c, (size_t)m, sizeof(scored_t), by_score_desc_then_index);
+  int n = m < k ? m : k;
+  unsigned char* chosen = (unsigned char*)calloc((size_t)(t + 1), 1);
+  for (int i = 0; i < n; ++i) chosen[c[i].s] = 1;
+  int wpos = 0;
+  for (int s = 0; s <= t; ++s)
+    if (chosen[s]) idx[wpos++] = s;
+  for (int i = n; i < k; ++i) idx[i] = -1;
+  free(chosen);
+  free(c);
+  free(one);
+  free(sc);
+  free(bsel);
+  free(mean);
+  free(bscore);
+  return n;
 }
 
 /* ---- f2: gradient of the indexer loss with respect to the indexer's inputs -------------- */

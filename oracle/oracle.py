@@ -49,6 +49,11 @@ def _load():
         lib.ref_dense_p_row.argtypes = [vp, vp, i32, i32, i32, f64, vp]
         lib.ref_dense_kl_row.argtypes = [vp, i32, vp]
         lib.ref_dense_kl_row.restype = f64
+        lib.ref_block_mean.argtypes = [vp, i32, i32, i32, vp]
+        lib.ref_block_score.argtypes = [vp, vp, vp, i32, i32]
+        lib.ref_block_score.restype = f64
+        lib.ref_hisa_row.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, vp, vp]
+        lib.ref_hisa_row.restype = i32
         lib.ref_indexer_loss_row_f64.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32]
         lib.ref_indexer_loss_row_f64.restype = f64
         lib.ref_indexer_grad_row.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, vp, vp, vp, vp]
@@ -151,6 +156,36 @@ def dense_kl_row(scores_row, t: int, p) -> float:
     scores_row, sp = _c(scores_row, np.float64)
     p, pp = _c(p, np.float64)
     return _load().ref_dense_kl_row(sp, t, pp)
+
+
+def block_mean(k_seq, s0: int, n: int) -> np.ndarray:
+    """Mean of the e4m3 keys [s0, s0+n) of k_seq [Lk, d_I]."""
+    k_seq, kp = _c(k_seq, np.uint8)
+    out = np.empty(k_seq.shape[1])
+    _load().ref_block_mean(kp, s0, n, k_seq.shape[1], out.ctypes.data)
+    return out
+
+
+def block_score(q_row, mean, w_row) -> float:
+    """sum_j w_j ReLU(q_j . mean) for e4m3 q_row [H_I, d_I] and a real mean key."""
+    q_row, qp = _c(q_row, np.uint8)
+    mean, mp = _c(mean, np.float64)
+    w_row, wp = _c(w_row, np.float32)
+    H_I, d_I = q_row.shape
+    return _load().ref_block_score(qp, mp, wp, H_I, d_I)
+
+
+def hisa_row(q_row, k_seq, w_row, t: int, bsize: int, r: int, k: int):
+    """HISA's selection for query t: (idx [k] ascending, -1 padded; kept blocks [r]; |S|)."""
+    q_row, qp = _c(q_row, np.uint8)
+    k_seq, kp = _c(k_seq, np.uint8)
+    w_row, wp = _c(w_row, np.float32)
+    H_I, d_I = q_row.shape
+    idx = np.empty(k, dtype=np.int32)
+    blocks = np.empty(r, dtype=np.int32)
+    n = _load().ref_hisa_row(qp, kp, wp, k_seq.shape[0], t, H_I, d_I, bsize, r, k, idx.ctypes.data,
+                             blocks.ctypes.data)
+    return idx, blocks, n
 
 
 def indexer_loss_row_f64(q_row, k_seq, w_row, idx, p) -> float:
