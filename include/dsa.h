@@ -156,6 +156,32 @@ dsa_status dsa_sparse_mla_fwd_paged(const void* q_bf16, const void* kv_pages, co
                                     size_t ws_bytes, dsa_stream_t stream);
 
 /*
+ * HISA, block -> token retrieval for decode ("DeepSeek-V3.2" analysis page, sec. 5.3: a coarse
+ * stage over block representatives, then exact indexer scores inside the kept blocks; cost
+ * model eq. (25), recall decomposition eq. (24)).  The cache of each sequence is cut into blocks
+ * of `block` keys (Lk a multiple of block).  A block is represented by the mean of its keys and
+ * scored with the indexer's formula on that mean key, sum_j w_j ReLU(q_I[b,j,:] . mean); the r
+ * blocks with the largest scores are kept (ties -> smaller block); every key in them gets its
+ * exact score (eq. (1)) and idx holds the min(k, r*block) best of those keys (ties -> smaller
+ * position), ascending, -1 padded.  With r * block >= Lk this is exactly dsa_indexer_topk's set.
+ *
+ * dsa_hisa_block_sums: the cache summary, computed once when the cache is written:
+ *   k_fp8 [B,Lk,d_I] e4m3 -> sums [B, ceil(Lk/block), d_I] fp32 (the sums of each block's keys).
+ * dsa_hisa_topk: one decode step's selection:
+ *   q_fp8 [B,1,H_I,d_I] e4m3, k_fp8 [B,Lk,d_I] e4m3, w [B,1,H_I] fp32, block_sums from above,
+ *   idx [B,1,k] int32 (output), blocks [B,1,r] int32 (nullable output: the kept blocks, ascending,
+ *   -1 padded when Lk / block < r),
+ *   ws: dsa_hisa_workspace_bytes(B, Lk, block, r, k) bytes.
+ * Supported: d_I = 128, H_I in {64, 32}, k <= 4096, r <= 4096, r * block <= 262144.
+ */
+size_t dsa_hisa_workspace_bytes(int B, int Lk, int block, int r, int k);
+dsa_status dsa_hisa_block_sums(const void* k_fp8, int B, int Lk, int d_I, int block, float* sums,
+                               dsa_stream_t stream);
+dsa_status dsa_hisa_topk(const void* q_fp8, const void* k_fp8, const float* w, const float* block_sums,
+                         int B, int Lk, int H_I, int d_I, int block, int r, int k, int32_t* idx,
+                         int32_t* blocks, void* ws, size_t ws_bytes, dsa_stream_t stream);
+
+/*
  * Sparse attention in MLA's MQA mode over the selected latents ("DeepSeek-V3.2" analysis
  * page, sec. 1.1, eq. (2) and the MQA-mode paragraph; renormalised form eq. (19)).
  * Every query head shares the latent entry c_s = kv[b,s,:]; keys use all d_qk dims,

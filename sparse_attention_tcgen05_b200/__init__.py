@@ -20,7 +20,7 @@ __all__ = [
     "dsa_topk", "dsa_sparse_mla_fwd", "dsa_indexer_kl", "dsa_indexer_kl_noalloc",
     "dsa_last_device_status", "dsa_set_wait_limit_ns", "dsa_selftest_wait", "dsa_dense_mla_fwd",
     "dsa_indexer_kl_dense", "dsa_indexer_topk", "dsa_indexer_bwd", "dsa_indexer_topk_paged",
-    "dsa_sparse_mla_fwd_paged",
+    "dsa_sparse_mla_fwd_paged", "dsa_hisa_workspace_bytes", "dsa_hisa_block_sums", "dsa_hisa_topk",
     "DSA_OP_INDEXER", "DSA_OP_TOPK", "DSA_OP_SPARSE_MLA_FWD", "DSA_OP_INDEXER_KL",
     "DSA_OP_DENSE_MLA_FWD", "DSA_OP_INDEXER_KL_DENSE", "DSA_OP_INDEXER_TOPK", "EXPORTED",
 ]
@@ -31,7 +31,8 @@ EXPORTED = ("dsa_status_str", "dsa_version", "dsa_workspace_bytes", "dsa_indexer
             "dsa_sparse_mla_fwd", "dsa_indexer_kl", "dsa_indexer_kl_noalloc",
             "dsa_last_device_status", "dsa_set_wait_limit_ns", "dsa_selftest_wait",
             "dsa_dense_mla_fwd", "dsa_indexer_kl_dense", "dsa_indexer_topk", "dsa_indexer_bwd",
-            "dsa_indexer_topk_paged", "dsa_sparse_mla_fwd_paged")
+            "dsa_indexer_topk_paged", "dsa_sparse_mla_fwd_paged", "dsa_hisa_workspace_bytes",
+            "dsa_hisa_block_sums", "dsa_hisa_topk")
 
 
 class DsaError(RuntimeError):
@@ -74,10 +75,15 @@ def load(rebuild: bool = False) -> ctypes.CDLL:
                                                sz, vp]
         lib.dsa_sparse_mla_fwd_paged.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, f32,
                                                  vp, vp, vp, sz, vp]
+        lib.dsa_hisa_workspace_bytes.argtypes = [i32, i32, i32, i32, i32]
+        lib.dsa_hisa_workspace_bytes.restype = sz
+        lib.dsa_hisa_block_sums.argtypes = [vp, i32, i32, i32, i32, vp, vp]
+        lib.dsa_hisa_topk.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, vp, vp, vp, sz, vp]
         for name in ("dsa_indexer", "dsa_topk", "dsa_sparse_mla_fwd", "dsa_indexer_kl",
                      "dsa_indexer_kl_noalloc", "dsa_last_device_status", "dsa_set_wait_limit_ns",
                      "dsa_selftest_wait", "dsa_dense_mla_fwd", "dsa_indexer_kl_dense", "dsa_indexer_topk",
-                     "dsa_indexer_bwd", "dsa_indexer_topk_paged", "dsa_sparse_mla_fwd_paged"):
+                     "dsa_indexer_bwd", "dsa_indexer_topk_paged", "dsa_sparse_mla_fwd_paged",
+                     "dsa_hisa_block_sums", "dsa_hisa_topk"):
             getattr(lib, name).restype = i32
         _lib = lib
     return _lib
@@ -322,6 +328,39 @@ def dsa_sparse_mla_fwd_paged(q: torch.Tensor, kv_pages: torch.Tensor, idx: torch
            load().dsa_sparse_mla_fwd_paged(_ptr(q), _ptr(kv_pages), _ptr(idx), _ptr(block_table), _ptr(seq_lens), B,
                                            max_len, num_pages, page_size, H, d_qk, d_v, k, float(scale), _ptr(out),
                                            _ptr(lse), wsp, wsb, _stream(stream)))
+
+
+def dsa_hisa_workspace_bytes(B: int, Lk: int, block: int, r: int, k: int) -> int:
+    return int(load().dsa_hisa_workspace_bytes(B, Lk, block, r, k))
+
+
+def dsa_hisa_block_sums(k_fp8: torch.Tensor, block: int, sums: torch.Tensor, stream=None) -> None:
+    """Per-block key sums of a k_I cache [B, Lk, d_I] e4m3 -> sums [B, ceil(Lk/block), d_I] fp32."""
+    B, Lk, d_I = k_fp8.shape
+    _check(k_fp8, "k_fp8", torch.float8_e4m3fn, (B, Lk, d_I))
+    _check(sums, "sums", torch.float32, (B, -(-Lk // block), d_I))
+    _raise("dsa_hisa_block_sums",
+           load().dsa_hisa_block_sums(_ptr(k_fp8), B, Lk, d_I, block, _ptr(sums), _stream(stream)))
+
+
+def dsa_hisa_topk(q_fp8: torch.Tensor, k_fp8: torch.Tensor, w: torch.Tensor, sums: torch.Tensor, block: int,
+                  r: int, idx: torch.Tensor, blocks: torch.Tensor | None = None, ws: torch.Tensor | None = None,
+                  stream=None) -> None:
+    """HISA decode selection: the r best blocks by their mean key, then the exact top-k inside."""
+    B, Lq, H_I, d_I = q_fp8.shape
+    Lk = k_fp8.shape[1]
+    k = idx.shape[2]
+    _check(q_fp8, "q_fp8", torch.float8_e4m3fn, (B, 1, H_I, d_I))
+    _check(k_fp8, "k_fp8", torch.float8_e4m3fn, (B, Lk, d_I))
+    _check(w, "w", torch.float32, (B, 1, H_I))
+    _check(sums, "sums", torch.float32, (B, -(-Lk // block), d_I))
+    _check(idx, "idx", torch.int32, (B, 1, k))
+    if blocks is not None:
+        _check(blocks, "blocks", torch.int32, (B, 1, r))
+    wsp, wsb = _ws(ws)
+    _raise("dsa_hisa_topk",
+           load().dsa_hisa_topk(_ptr(q_fp8), _ptr(k_fp8), _ptr(w), _ptr(sums), B, Lk, H_I, d_I, block, r, k,
+                                _ptr(idx), _ptr(blocks), wsp, wsb, _stream(stream)))
 
 
 def dsa_indexer_kl_noalloc(scores: torch.Tensor, idx: torch.Tensor, p_sel: torch.Tensor,

@@ -12,6 +12,7 @@
 #include <utility>
 
 #include "../../include/dsa.h"
+#include "hisa.cuh"
 #include "indexer.cuh"
 #include "indexer_bwd.cuh"
 #include "indexer_kl.cuh"
@@ -429,6 +430,32 @@ __global__ void wait_selftest_kernel() {
   dsa::mbar_wait(&bar, 0, &abort_flag, 90);
 }
 
+// ------------------------------------------------------------------------------ HISA workspace
+struct HisaWs {  // workspace regions of dsa_hisa_topk (each 256-byte aligned)
+  size_t bscores, bidx, pages, seq, cscores, cidx, hist, total;
+};
+inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+HisaWs hisa_ws(int B, int Lk, int block, int r, int k) {
+  HisaWs w{};
+  const size_t nb = static_cast<size_t>((Lk + block - 1) / block);
+  size_t o = 0;
+  w.bscores = o; o = align256(o + static_cast<size_t>(B) * nb * 4);
+  w.bidx = o;    o = align256(o + static_cast<size_t>(B) * r * 4);
+  w.pages = o;   o = align256(o + static_cast<size_t>(B) * r * 4);
+  w.seq = o;     o = align256(o + static_cast<size_t>(B) * 4);
+  w.cscores = o; o = align256(o + static_cast<size_t>(B) * r * block * 4);
+  w.cidx = o;    o = align256(o + static_cast<size_t>(B) * k * 4);
+  w.hist = o;    o = align256(o + static_cast<size_t>(B) * 2048 * 4);
+  w.total = o;
+  return w;
+}
+
+__global__ void hisa_seq_lens_kernel(int32_t* seq, int B, int n) {
+  dsa::pdl_launch_dependents();
+  dsa::pdl_wait();
+  for (int b = blockIdx.x * blockDim.x + threadIdx.x; b < B; b += gridDim.x * blockDim.x) seq[b] = n;
+}
+
 }  // namespace
 
 // ================================================================================ C ABI
@@ -762,6 +789,86 @@ dsa_status dsa_sparse_mla_fwd_paged(const void* q_bf16, const void* kv_pages, co
   if (ds != DSA_OK) return ds;
   return launch_mla<576, 512>(q_bf16, kv_pages, idx, B, 1, max_len, H, k, scale, out_bf16, lse, nullptr, ws, ws_bytes,
                               dev.sms, static_cast<cudaStream_t>(stream), 0, &pg);
+}
+
+
+size_t dsa_hisa_workspace_bytes(int B, int Lk, int block, int r, int k) {
+  if (B <= 0 || Lk <= 0 || block <= 0 || r <= 0 || k <= 0) return 0;
+  return hisa_ws(B, Lk, block, r, k).total;
+}
+
+dsa_status dsa_hisa_block_sums(const void* k_fp8, int B, int Lk, int d_I, int block, float* sums,
+                                          dsa_stream_t stream) {
+  if (!k_fp8 || !sums || B <= 0 || Lk <= 0 || block <= 0 || d_I <= 0) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(k_fp8) || !aligned16(sums)) return DSA_ERR_INVALID_ARG;
+  if (d_I != dsa::hisa::kDI) return DSA_ERR_UNSUPPORTED;
+  const long n_blocks = (Lk + block - 1) / block;
+  if (static_cast<long>(B) * n_blocks > INT32_MAX || static_cast<long>(B) * Lk >= INT32_MAX) return DSA_ERR_UNSUPPORTED;
+  DeviceInfo dev;
+  const dsa_status ds = current_device(dev);
+  if (ds != DSA_OK) return ds;
+  return launch(dsa::hisa::block_sums_kernel, static_cast<unsigned>(B * n_blocks), dsa::hisa::kSumThreads, 0,
+                static_cast<cudaStream_t>(stream), 1, static_cast<const uint8_t*>(k_fp8), Lk, block,
+                static_cast<int>(n_blocks), sums);
+}
+
+dsa_status dsa_hisa_topk(const void* q_fp8, const void* k_fp8, const float* w, const float* block_sums,
+                                    int B, int Lk, int H_I, int d_I, int block, int r, int k, int32_t* idx,
+                                    int32_t* blocks, void* ws, size_t ws_bytes, dsa_stream_t stream) {
+  if (!q_fp8 || !k_fp8 || !w || !block_sums || !idx || !ws) return DSA_ERR_INVALID_ARG;
+  if (B <= 0 || Lk <= 0 || block <= 0 || r <= 0 || k <= 0) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q_fp8) || !aligned16(k_fp8) || !aligned16(w) || !aligned16(block_sums) || !aligned16(idx) ||
+      (blocks && !aligned16(blocks)) || !aligned16(ws))
+    return DSA_ERR_INVALID_ARG;
+  if (Lk % block != 0) return DSA_ERR_UNSUPPORTED;  // the cache is whole blocks
+  if (!fused_topk_shape(1, H_I, d_I)) return DSA_ERR_UNSUPPORTED;
+  const int n_blocks = Lk / block;
+  const int r_eff = std::min(r, n_blocks);
+  if (k > 4096 || r > 4096 || static_cast<long>(r) * block > 262144 || n_blocks > 262144) return DSA_ERR_UNSUPPORTED;
+  if (static_cast<long>(B) * Lk >= INT32_MAX) return DSA_ERR_UNSUPPORTED;
+  const HisaWs L = hisa_ws(B, Lk, block, r, k);
+  if (ws_bytes < L.total) return DSA_ERR_INVALID_ARG;
+  DeviceInfo dev;
+  const dsa_status ds = current_device(dev);
+  if (ds != DSA_OK) return ds;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  float* bscores = reinterpret_cast<float*>(base + L.bscores);
+  int32_t* bidx = blocks ? blocks : reinterpret_cast<int32_t*>(base + L.bidx);
+  int32_t* pages = reinterpret_cast<int32_t*>(base + L.pages);
+  int32_t* seq = reinterpret_cast<int32_t*>(base + L.seq);
+  float* cscores = reinterpret_cast<float*>(base + L.cscores);
+  int32_t* cidx = reinterpret_cast<int32_t*>(base + L.cidx);
+  uint32_t* hist = reinterpret_cast<uint32_t*>(base + L.hist);
+  // 1. coarse scores of every block; 2. the r best blocks (ascending)
+  const dim3 sgrid(static_cast<unsigned>(B), static_cast<unsigned>((n_blocks + dsa::hisa::kScoreThreads - 1) /
+                                                                    dsa::hisa::kScoreThreads));
+  if (H_I == 64)
+    dsa::hisa::block_scores_kernel<64><<<sgrid, dsa::hisa::kScoreThreads, 0, st>>>(
+        static_cast<const uint8_t*>(q_fp8), w, block_sums, Lk, block, n_blocks, bscores);
+  else
+    dsa::hisa::block_scores_kernel<32><<<sgrid, dsa::hisa::kScoreThreads, 0, st>>>(
+        static_cast<const uint8_t*>(q_fp8), w, block_sums, Lk, block, n_blocks, bscores);
+  if (launch_result() != DSA_OK) return DSA_ERR_CUDA;
+  dsa_status s = run_topk(bscores, bidx, B, 1, n_blocks, r, dev.sms, st, nullptr);
+  if (s != DSA_OK) return s;
+  // 3. the kept blocks as the pages of the exact stage, every candidate slot valid
+  s = launch(dsa::hisa::block_pages_kernel, static_cast<unsigned>(B), 128u, 0, st, 1,
+             static_cast<const int32_t*>(bidx), r, n_blocks, pages);
+  if (s != DSA_OK) return s;
+  s = launch(hisa_seq_lens_kernel, static_cast<unsigned>((B + 255) / 256), 256u, 0, st, 1, seq, B, r_eff * block);
+  if (s != DSA_OK) return s;
+  // 4. exact indexer scores on the candidates and their top-k (the paged decode path)
+  Paging pg{pages, seq, block, r, B * n_blocks};
+  if (cudaMemsetAsync(hist, 0, static_cast<size_t>(B) * 2048 * sizeof(uint32_t), st) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  s = run_indexer(q_fp8, k_fp8, w, cscores, B, 1, r * block, H_I, d_I, dev.sms, st, hist, &pg);
+  if (s != DSA_OK) return s;
+  s = run_topk(cscores, cidx, B, 1, r * block, k, dev.sms, st, hist, seq);
+  if (s != DSA_OK) return s;
+  // 5. candidate slots -> positions
+  return launch(dsa::hisa::slots_to_positions_kernel, static_cast<unsigned>(B), 256u, 0, st, 1,
+                static_cast<const int32_t*>(cidx), static_cast<const int32_t*>(bidx), r, block, k, idx);
 }
 
 dsa_status dsa_set_wait_limit_ns(uint64_t ns) {
