@@ -317,8 +317,11 @@ class Step:
         pk = Lk if wl.dense else wl.k  # the dense target covers every position
         self.p = torch.empty(B, Lq, pk, dtype=torch.float32, device=device) if wl.emit_p else None
         self.loss = torch.empty(1, dtype=torch.float32, device=device)
+        # the fused decode indexer -> top-k keeps its histograms zero-filled between calls: a
+        # buffer of its own, cleared once
+        self.ws_ix = torch.zeros(max(16, dsa.dsa_workspace_bytes(dsa.DSA_OP_INDEXER_TOPK, B, Lq, Lk, wl.k, 0)),
+                                 dtype=torch.uint8, device=device)
         nws = max(dsa.dsa_workspace_bytes(dsa.DSA_OP_SPARSE_MLA_FWD, B, Lq, Lk, wl.k, wl.H),
-                  dsa.dsa_workspace_bytes(dsa.DSA_OP_INDEXER_TOPK, B, Lq, Lk, wl.k, 0),
                   dsa.dsa_workspace_bytes(dsa.DSA_OP_DENSE_MLA_FWD, B, Lq, Lk, 0, wl.H) if wl.dense else 0,
                   dsa.dsa_workspace_bytes(dsa.DSA_OP_INDEXER_KL, B, Lq, Lk, wl.k, 0), 16)
         self.ws = torch.empty(nws, dtype=torch.uint8, device=device)
@@ -345,7 +348,7 @@ class Step:
         if ev:
             ev[0].record()
         if wl.Lq == 1 and not wl.dense:  # decode: the fused indexer -> top-k (one stage)
-            dsa.dsa_indexer_topk(d["qI"], d["kI"], d["w"], self.scores, self.idx, self.ws)
+            dsa.dsa_indexer_topk(d["qI"], d["kI"], d["w"], self.scores, self.idx, self.ws_ix)
             if ev:
                 ev[1].record()
                 ev[2].record()

@@ -113,7 +113,11 @@ dsa_status dsa_topk(const float* scores, int32_t* idx, int B, int Lq, int Lk, in
  * among the indexer's constant-factor savings, sec. 5.2 closing paragraph; decode step cost of
  * sec. 5.3, eq. (23)).
  *   ws: dsa_workspace_bytes(DSA_OP_INDEXER_TOPK, B, Lq, Lk, k, 0) bytes (the per-row histograms,
- *       B * Lq * 8 KiB for decode, 0 otherwise); it is cleared on the stream by the call itself.
+ *       B * Lq * 8 KiB for decode, 0 otherwise).  It must be zero-filled before its first use
+ *       (e.g. one cudaMemset); every call whose kernels complete leaves it zero-filled again, so
+ *       no clearing is needed between calls.  After a call that fails on the device (a status
+ *       other than DSA_OK from dsa_last_device_status) clear it again.  Calls that share one ws
+ *       must not overlap on the GPU.
  * Supported: the union of dsa_indexer's and dsa_topk's limits.
  */
 dsa_status dsa_indexer_topk(const void* q_fp8, const void* k_fp8, const float* w, float* scores,
@@ -133,8 +137,10 @@ dsa_status dsa_indexer_topk(const void* q_fp8, const void* k_fp8, const float* w
  *   are clamped and a page index outside [0, num_pages) reads as an empty entry, both recorded
  *   as DSA_ERR_INVALID_ARG in the device status word)
  *   scores [B,1,max_len] fp32 (-inf for s >= seq_lens[b]), idx [B,1,k] int32
- *   ws: dsa_workspace_bytes(DSA_OP_INDEXER_TOPK, B, 1, max_len, k, 0) bytes
- * Supported: (H_I, d_I) in {(64, 128), (32, 128)}, k <= 4096, max_len <= 262144.
+ *   ws: dsa_workspace_bytes(DSA_OP_INDEXER_TOPK, B, 1, max_len, k, 0) bytes, zero-filled before
+ *   its first use and left so by every call (as for dsa_indexer_topk)
+ * Supported: page_size a multiple of 64, (H_I, d_I) in {(64, 128), (32, 128)}, k <= 4096,
+ * max_len <= 262144.
  */
 dsa_status dsa_indexer_topk_paged(const void* q_fp8, const void* k_pages, const float* w,
                                   const int32_t* block_table, const int32_t* seq_lens, float* scores,
@@ -147,7 +153,7 @@ dsa_status dsa_indexer_topk_paged(const void* q_fp8, const void* k_pages, const 
  *   q_bf16 [B,1,H,576] bf16, kv_pages [num_pages,page_size,576] bf16, idx [B,1,k] int32
  *   (positions within each sequence), out_bf16 [B,1,H,512], lse [B,1,H] (nullable)
  *   ws: dsa_workspace_bytes(DSA_OP_SPARSE_MLA_FWD, B, 1, max_len, k, H) bytes
- * Supported: (d_qk, d_v) = (576, 512), H <= 128, k <= 65536.
+ * Supported: page_size a multiple of 64, (d_qk, d_v) = (576, 512), H <= 128, k <= 65536.
  */
 dsa_status dsa_sparse_mla_fwd_paged(const void* q_bf16, const void* kv_pages, const int32_t* idx,
                                     const int32_t* block_table, const int32_t* seq_lens, int B,
@@ -171,8 +177,10 @@ dsa_status dsa_sparse_mla_fwd_paged(const void* q_bf16, const void* kv_pages, co
  *   q_fp8 [B,1,H_I,d_I] e4m3, k_fp8 [B,Lk,d_I] e4m3, w [B,1,H_I] fp32, block_sums from above,
  *   idx [B,1,k] int32 (output), blocks [B,1,r] int32 (nullable output: the kept blocks, ascending,
  *   -1 padded when Lk / block < r),
- *   ws: dsa_hisa_workspace_bytes(B, Lk, block, r, k) bytes.
- * Supported: d_I = 128, H_I in {64, 32}, k <= 4096, r <= 4096, r * block <= 262144.
+ *   ws: dsa_hisa_workspace_bytes(B, Lk, block, r, k) bytes, zero-filled before its first use
+ *   and left so by every call (its histograms are those of dsa_indexer_topk).
+ * Supported: block a multiple of 64, d_I = 128, H_I in {64, 32}, k <= 4096, r <= 4096,
+ * r * block <= 262144.
  */
 size_t dsa_hisa_workspace_bytes(int B, int Lk, int block, int r, int k);
 dsa_status dsa_hisa_block_sums(const void* k_fp8, int B, int Lk, int d_I, int block, float* sums,

@@ -160,10 +160,11 @@ dsa_status launch_indexer(const void* q, const void* kk, const float* w, float* 
                  D_I, D_I, Cfg::N, swz))
     return DSA_ERR_CUDA;
   const uint64_t k_rows = pg ? static_cast<uint64_t>(pg->num_pages) * pg->page_size : static_cast<uint64_t>(B) * Lk;
-  if (!encode_2d(&tm_k, CU_TENSOR_MAP_DATA_TYPE_UINT8, kk, D_I, k_rows, D_I, D_I, dsa::indexer::kTileKeys, swz))
+  if (k_rows >= INT32_MAX) return DSA_ERR_UNSUPPORTED;
+  if (!encode_2d(&tm_k, CU_TENSOR_MAP_DATA_TYPE_UINT8, kk, D_I, k_rows, D_I, D_I, Cfg::kKBox, swz))
     return DSA_ERR_CUDA;
   dsa::indexer::Params p{};
-  p.k = static_cast<const uint8_t*>(kk);
+  p.k_rows = static_cast<int>(k_rows);
   if (pg) {
     p.block_table = pg->block_table;
     p.seq_lens = pg->seq_lens;
@@ -203,7 +204,7 @@ dsa_status launch_indexer(const void* q, const void* kk, const float* w, float* 
 // ------------------------------------------------------------------------------ top-k
 template <int C, int KPT>
 dsa_status launch_topk(const float* scores, int32_t* idx, int B, int Lq, int Lk, int k,
-                       cudaStream_t stream, const uint32_t* ghist, const int32_t* seq_lens) {
+                       cudaStream_t stream, uint32_t* ghist, const int32_t* seq_lens) {
   auto kern = dsa::topk::topk_kernel<C, KPT>;
   constexpr int smem = dsa::topk::dyn_smem_bytes<KPT>();
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
@@ -225,7 +226,7 @@ int topk_cluster_size(int rows, int Lk, int sms) {
 
 template <int C>
 dsa_status launch_topk_c(const float* scores, int32_t* idx, int B, int Lq, int Lk, int k,
-                         cudaStream_t st, const uint32_t* ghist, const int32_t* sl) {
+                         cudaStream_t st, uint32_t* ghist, const int32_t* sl) {
   const int slice = topk_slice(Lk, C);
   if (slice <= 4 * dsa::topk::kThreads) return launch_topk<C, 4>(scores, idx, B, Lq, Lk, k, st, ghist, sl);
   if (slice <= 8 * dsa::topk::kThreads) return launch_topk<C, 8>(scores, idx, B, Lq, Lk, k, st, ghist, sl);
@@ -236,7 +237,7 @@ dsa_status launch_topk_c(const float* scores, int32_t* idx, int B, int Lq, int L
 // Top-k with the validated sizes; ghist (nullable) holds each row's top-digit counts, seq_lens
 // (nullable, Lq == 1) each row's context length.
 dsa_status run_topk(const float* scores, int32_t* idx, int B, int Lq, int Lk, int k, int sms, cudaStream_t st,
-                    const uint32_t* ghist, const int32_t* seq_lens = nullptr) {
+                    uint32_t* ghist, const int32_t* seq_lens = nullptr) {
   switch (topk_cluster_size(B * Lq, Lk, sms)) {
     case 1: return launch_topk_c<1>(scores, idx, B, Lq, Lk, k, st, ghist, seq_lens);
     case 2: return launch_topk_c<2>(scores, idx, B, Lq, Lk, k, st, ghist, seq_lens);
@@ -554,8 +555,7 @@ dsa_status dsa_indexer_topk(const void* q_fp8, const void* k_fp8, const float* w
   const dsa_status ds = current_device(dev);
   if (ds != DSA_OK) return ds;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  uint32_t* hist = fused ? static_cast<uint32_t*>(ws) : nullptr;
-  if (fused && cudaMemsetAsync(hist, 0, need, st) != cudaSuccess) return DSA_ERR_CUDA;
+  uint32_t* hist = fused ? static_cast<uint32_t*>(ws) : nullptr;  // zero-filled between calls
   const dsa_status si = run_indexer(q_fp8, k_fp8, w, scores, B, Lq, Lk, H_I, d_I, dev.sms, st, hist);
   if (si != DSA_OK) return si;
   return run_topk(scores, idx, B, Lq, Lk, k, dev.sms, st, hist);
@@ -737,6 +737,7 @@ dsa_status check_paging(const int32_t* block_table, const int32_t* seq_lens, int
   if (!block_table || !seq_lens) return DSA_ERR_INVALID_ARG;
   if (B <= 0 || max_len <= 0 || num_pages <= 0 || page_size <= 0) return DSA_ERR_INVALID_ARG;
   if (!aligned16(block_table) || !aligned16(seq_lens)) return DSA_ERR_INVALID_ARG;
+  if (page_size % 64 != 0) return DSA_ERR_UNSUPPORTED;  // the indexer loads pages in boxes of 64 keys
   if (static_cast<long>(num_pages) * page_size >= INT32_MAX || static_cast<long>(B) * max_len >= INT32_MAX)
     return DSA_ERR_UNSUPPORTED;
   pg->block_table = block_table;
@@ -765,8 +766,7 @@ dsa_status dsa_indexer_topk_paged(const void* q_fp8, const void* k_pages, const 
   const dsa_status ds = current_device(dev);
   if (ds != DSA_OK) return ds;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  uint32_t* hist = static_cast<uint32_t*>(ws);
-  if (cudaMemsetAsync(hist, 0, need, st) != cudaSuccess) return DSA_ERR_CUDA;
+  uint32_t* hist = static_cast<uint32_t*>(ws);  // zero-filled between calls
   const dsa_status si = run_indexer(q_fp8, k_pages, w, scores, B, 1, max_len, H_I, d_I, dev.sms, st, hist, &pg);
   if (si != DSA_OK) return si;
   return run_topk(scores, idx, B, 1, max_len, k, dev.sms, st, hist, seq_lens);
@@ -820,7 +820,7 @@ dsa_status dsa_hisa_topk(const void* q_fp8, const void* k_fp8, const float* w, c
   if (!aligned16(q_fp8) || !aligned16(k_fp8) || !aligned16(w) || !aligned16(block_sums) || !aligned16(idx) ||
       (blocks && !aligned16(blocks)) || !aligned16(ws))
     return DSA_ERR_INVALID_ARG;
-  if (Lk % block != 0) return DSA_ERR_UNSUPPORTED;  // the cache is whole blocks
+  if (Lk % block != 0 || block % 64 != 0) return DSA_ERR_UNSUPPORTED;  // whole blocks, loaded 64 keys at a time
   if (!fused_topk_shape(1, H_I, d_I)) return DSA_ERR_UNSUPPORTED;
   const int n_blocks = Lk / block;
   const int r_eff = std::min(r, n_blocks);
@@ -859,9 +859,7 @@ dsa_status dsa_hisa_topk(const void* q_fp8, const void* k_fp8, const float* w, c
   s = launch(hisa_seq_lens_kernel, static_cast<unsigned>((B + 255) / 256), 256u, 0, st, 1, seq, B, r_eff * block);
   if (s != DSA_OK) return s;
   // 4. exact indexer scores on the candidates and their top-k (the paged decode path)
-  Paging pg{pages, seq, block, r, B * n_blocks};
-  if (cudaMemsetAsync(hist, 0, static_cast<size_t>(B) * 2048 * sizeof(uint32_t), st) != cudaSuccess)
-    return DSA_ERR_CUDA;
+  Paging pg{pages, seq, block, r, B * n_blocks};  // hist: zero-filled between calls
   s = run_indexer(q_fp8, k_fp8, w, cscores, B, 1, r * block, H_I, d_I, dev.sms, st, hist, &pg);
   if (s != DSA_OK) return s;
   s = run_topk(cscores, cidx, B, 1, r * block, k, dev.sms, st, hist, seq);

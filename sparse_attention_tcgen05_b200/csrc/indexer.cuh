@@ -8,11 +8,10 @@
 //
 // Persistent, warp-specialised CTA (one per SM):
 //   warp 0        TMA producer: the q_I group once per work item, then k_I tiles (12 stages
-//                 for decode, 6 otherwise).  For decode (one query per tile, a pure stream of
-//                 k_I) warps 0 and 2 load the k_I tiles with 16-byte cp.async copies written
-//                 straight into the 128B-swizzled layout instead, and warp 3 loads the q_I
-//                 groups: plain loads stream from HBM faster than TMA tile copies on B200 (about
-//                 6.0 against 5.5 TB/s for a 512 MiB read), and decode is bound by that stream.
+//                 for decode, 6 otherwise).  Decode loads each 128-key tile as two boxes of 64
+//                 keys (so that a paged cache can place them in different pages) and marks k_I
+//                 evict-first in L2: it is read once, and the scores written meanwhile should stay
+//                 there for the top-k.
 //   warp 1        MMA issuer (one thread): d_I/32 MMAs of 128 x N x 32 per tile
 //   warp 2        TMEM allocator (2 accumulators of N columns, double-buffered)
 //   warps 4..11   epilogue: tcgen05.ld -> ReLU * w -> head sum -> mask -> store; for decode
@@ -36,7 +35,6 @@ constexpr int kThreads = 128 + kEpiWarps * 32;
 constexpr int kTileKeys = 128;
 
 struct Params {
-  const uint8_t* k;  // k_I [B * Lk, d_I] (the decode loads read it directly)
   const float* w;
   float* scores;
   uint32_t* hist;    // nullable, decode only: [B * Lq][2048] counts of the scores' top digit
@@ -45,7 +43,8 @@ struct Params {
   // sits at t = seq_lens[b] - 1 (clamped to [-1, Lk - 1]; Lk is then the longest context).
   const int32_t* block_table;
   const int32_t* seq_lens;
-  int page_size, max_pages, num_pages;
+  int page_size, max_pages, num_pages;  // page_size: a multiple of 64
+  int k_rows;                           // rows of the k tensor (one past it reads as zeros)
   int B, Lq, Lk;
   int n_qg;   // query groups per sequence
   int n_kt;   // key tiles per sequence
@@ -54,18 +53,12 @@ struct Params {
   int n_items;
 };
 
-// Decode k_I producers (cp.async): warps 0 and 2, and how many tiles each keeps in flight
-// before it signals the oldest one.
-constexpr int kLoadThreads = 64;
-constexpr int kLoadLag = 6;
-
 template <int H_I, int D_I, int G>
 struct Cfg {
   // k_I ring depth: decode streams k_I from HBM with little else per tile, so it keeps twice
   // as many tiles in flight
   static constexpr int kStages = (G == 1) ? 12 : 6;
-  static constexpr bool kCpAsyncK = (G == 1) && (D_I == 128);  // decode: k_I by cp.async
-  static_assert(!kCpAsyncK || kLoadLag < kStages, "the producer signals tile j - lag before reusing stage j");
+  static constexpr int kKBox = (G == 1) ? 64 : kTileKeys;  // keys per k_I TMA box
   static constexpr int N = G * H_I;                      // MMA N (columns per accumulator)
   static constexpr int kQBytes = N * D_I;                // q_I group tile
   static constexpr int kKBytes = kTileKeys * D_I;        // k_I tile
@@ -120,7 +113,8 @@ __device__ __forceinline__ void item_tiles(const Params& p, int b, int qg, int k
   n_comp = max(0, min(kt1, last_visible_tile + 1) - kt0);
 }
 
-// Row of k holding key s of sequence b (-1: no such key).
+// Row of k holding key s of sequence b (-1: a bad page index, recorded).  In a paged cache the 64
+// keys from a multiple of 64 lie in one page.
 __device__ __forceinline__ long key_row(const Params& p, int b, int s) {
   if (p.block_table == nullptr) return static_cast<long>(b) * p.Lk + s;
   const int page = __ldg(p.block_table + static_cast<size_t>(b) * p.max_pages + s / p.page_size);
@@ -162,7 +156,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
-      mbar_init(&k_full[s], C::kCpAsyncK ? kLoadThreads : 1);
+      mbar_init(&k_full[s], 1);
       mbar_init(&k_empty[s], 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -183,91 +177,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
   pdl_wait();  // first global access below
 
-  if (C::kCpAsyncK && warp == 3) {
-    // ------------------------------------------------------------------ decode: q_I groups
-    // A thread of its own: its wait for a free q_I buffer (item u - 2 consumed) must never hold
-    // back the k_I producers, which signal their tiles a few tiles late.
-    if (lane == 0) {
-      tma_prefetch_desc(&tm_q);
-      int qi = 0;
-      for (int u = blockIdx.x; u < p.n_items; u += gridDim.x) {
-        int b, qg, kc, kt0, kt1, n_comp;
-        decode_item(p, u, b, qg, kc);
-        item_tiles<G>(p, b, qg, kc, kt0, kt1, n_comp);
-        if (n_comp == 0) continue;
-        const int qb = qi & 1;
-        const uint32_t qph = (qi >> 1) & 1;
-        if (!mbar_wait(&q_empty[qb], qph ^ 1, abort_flag, 1)) break;
-        mbar_arrive_expect_tx(&q_full[qb], C::kQBytes);
-        tma_load_2d(sQ + qb * ((C::kQBytes + 1023) / 1024) * 1024, &tm_q, &q_full[qb], 0,
-                    (b * p.Lq + qg * G) * H_I);
-        ++qi;
-      }
-    }
-  } else if (C::kCpAsyncK && (warp == 0 || warp == 2)) {
-    // ------------------------------------------------------------------ decode: k_I tiles
-    // Thread pt of the 64 copies the 16-byte chunks pt, pt + 64, ... of a tile (consecutive
-    // threads read consecutive bytes), each to its 128B-swizzled place.  A thread signals tile
-    // j on the tile's barrier once its copies of tile j have landed (cp.async.wait_group) and are
-    // made visible to the tensor cores' async proxy, which it checks after issuing tile j + lag.
-    // No wait of these threads depends on a tile they have not signalled: tile j + kStages
-    // waits for tile j to be consumed, which needs only tiles <= j signalled (lag < stages) and
-    // the q_I group of tile j's item, loaded by warp 3 once the item two back is consumed.
-    const int pt = (warp == 0 ? 0 : 32) + lane;
-    const size_t k_rows = p.block_table ? static_cast<size_t>(p.num_pages) * p.page_size
-                                        : static_cast<size_t>(p.B) * p.Lk;
-    // k_I is read once: its lines go first out of L2, so that the scores written meanwhile stay
-    // there for the top-k that reads them next
-    const uint64_t evict_first = l2_evict_first_policy();
-    int ks = 0, sig = 0;  // stage of the next tile; stage of the oldest unsignalled tile
-    uint32_t kph = 0;
-    int pending = 0;      // tiles issued but not signalled by this thread
-    bool ok = true;
-    for (int u = blockIdx.x; ok && u < p.n_items; u += gridDim.x) {
-      int b, qg, kc, kt0, kt1, n_comp;
-      decode_item(p, u, b, qg, kc);
-      item_tiles<G>(p, b, qg, kc, kt0, kt1, n_comp);
-      for (int tt = 0; tt < n_comp; ++tt) {
-        if (!mbar_wait(&k_empty[ks], kph ^ 1, abort_flag, 2)) {
-          ok = false;
-          break;
-        }
-        const int s0 = (kt0 + tt) * kTileKeys;
-        const uint32_t dst = smem_u32(sK + ks * C::kKBytes);
-        for (int c = pt; c < kTileKeys * (D_I / 16); c += kLoadThreads) {
-          const int r = c >> 3, ch = c & 7;
-          // keys past the sequence (or past the tensor) are zero-filled
-          const long kr = s0 + r < p.Lk ? key_row(p, b, s0 + r) : -1;
-          const bool valid = kr >= 0 && static_cast<size_t>(kr) < k_rows;
-          cp_async_16_hint(dst + swizzled_offset(r, ch, 128), p.k + (valid ? static_cast<size_t>(kr) * D_I + ch * 16 : 0),
-                           valid, evict_first);
-        }
-        cp_async_commit();
-        if (++pending > kLoadLag) {
-          cp_async_wait_group<kLoadLag>();
-          fence_proxy_async_smem();
-          mbar_arrive(&k_full[sig]);
-          if (++sig == C::kStages) sig = 0;
-          --pending;
-        }
-        if (++ks == C::kStages) {
-          ks = 0;
-          kph ^= 1;
-        }
-      }
-    }
-    // the remaining tiles (also after an abort: nothing of ours may land after exit)
-    cp_async_wait_group<0>();
-    fence_proxy_async_smem();
-    for (; pending > 0; --pending) {
-      mbar_arrive(&k_full[sig]);
-      if (++sig == C::kStages) sig = 0;
-    }
-  } else if (warp == 0) {
+  if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
+      const uint64_t evict_first = l2_evict_first_policy();
       int ks = 0;
       uint32_t kph = 0;
       int qi = 0;
@@ -285,8 +200,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int tt = 0; tt < n_comp; ++tt) {
           if (!mbar_wait(&k_empty[ks], kph ^ 1, abort_flag, 2)) goto done;
           mbar_arrive_expect_tx(&k_full[ks], C::kKBytes);
-          tma_load_2d(sK + ks * C::kKBytes, &tm_k, &k_full[ks], 0,
-                      b * p.Lk + (kt0 + tt) * kTileKeys);
+          if constexpr (G == 1) {
+            // two boxes of 64 keys; a box past the query (or the sequence) is read as zeros from
+            // one row past the tensor, never through the page table
+            const int t_row = query_pos(p, b, qg);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int s0 = (kt0 + tt) * kTileKeys + h * C::kKBox;
+              const long y = s0 <= t_row ? key_row(p, b, s0) : -1;
+              tma_load_2d_hint(sK + ks * C::kKBytes + h * C::kKBox * D_I, &tm_k, &k_full[ks], 0,
+                               y >= 0 ? static_cast<int32_t>(y) : p.k_rows, evict_first);
+            }
+          } else {
+            tma_load_2d(sK + ks * C::kKBytes, &tm_k, &k_full[ks], 0, b * p.Lk + (kt0 + tt) * kTileKeys);
+          }
           if (++ks == C::kStages) {
             ks = 0;
             kph ^= 1;
@@ -399,8 +326,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (i < p.Lq) {
               const int t = query_pos(p, b, i);
               p.scores[(row_base + i) * p.Lk + s] = (s <= t) ? acc[g] : -INFINITY;
-              if (G == 1 && count && s <= t) atomicAdd(&sHist[ordered_key(acc[g]) >> 21], 1u);
             }
+          }
+        }
+        if constexpr (G == 1) {
+          if (count) {
+            // the tile's visible scores by top digit: one shared atomic per distinct digit and
+            // warp (integer-valued scores crowd into a few digits)
+            const int t = query_pos(p, b, i0);
+            const uint32_t bin = (s < p.Lk && s <= t) ? (ordered_key(acc[0]) >> 21) : 0xFFFFFFFFu;
+            const uint32_t peers = __match_any_sync(0xFFFFFFFFu, bin);
+            if (bin != 0xFFFFFFFFu && lane == __ffs(peers) - 1) atomicAdd(&sHist[bin], __popc(peers));
           }
         }
       }

@@ -8,7 +8,9 @@
 //   1. every CTA counts its keys by the top digit; the cluster's counts (summed through
 //      distributed shared memory, two bins per request) give the digit d1 that holds T.  When
 //      the indexer already counted the row's top digits (the fused decode path, `ghist`), that
-//      histogram gives d1 directly and this pass and its cluster round are skipped;
+//      histogram gives d1 directly and this pass and its cluster round are skipped; the row's
+//      histogram is cleared again once every CTA of the row has read it, so the buffer is all
+//      zeros between calls;
 //   2. the candidates - keys whose top digit is d1, usually a few thousand per row - are pushed
 //      with their positions into every CTA of the cluster, together with each CTA's count of
 //      keys above d1; after one cluster barrier every CTA settles the two lower digits on the
@@ -205,7 +207,7 @@ __device__ __forceinline__ uint2 block_exclusive2(uint32_t a, uint32_t b, uint32
 template <int C, int KPT>
 __global__ void __launch_bounds__(kThreads, 1)
     topk_kernel(const float* __restrict__ scores, int32_t* __restrict__ idx, int B, int Lq, int Lk,
-                int k, const uint32_t* __restrict__ ghist, const int32_t* __restrict__ seq_lens) {
+                int k, uint32_t* __restrict__ ghist, const int32_t* __restrict__ seq_lens) {
   static_assert(KPT == 4 || KPT == 8 || KPT == 16 || KPT == 32, "keys per thread");
   static_assert(C == 1 || C == 2 || C == 4 || C == kMaxCluster, "cluster size");
   constexpr int kCpr = KPT / 4;  // chunks per thread
@@ -235,6 +237,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (n <= k) {  // every visible position is selected
     pdl_wait();
     for (int x = rank * kThreads + tid; x < k; x += C * kThreads) out[x] = x < n ? x : -1;
+    if (ghist != nullptr && rank == 0)  // leave the row's histogram cleared
+      for (int x = tid; x < 2048; x += kThreads) ghist[static_cast<size_t>(row) * 2048 + x] = 0u;
     return;
   }
 
@@ -392,6 +396,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     cluster_barrier();  // every candidate and count has landed; nothing remote follows on the fast path
   else
     __syncthreads();
+  if (pre && rank == 0)  // every CTA of the row has read the row's histogram: clear it for the next call
+    for (int x = tid; x < 2048; x += kThreads) ghist[static_cast<size_t>(row) * 2048 + x] = 0u;
 
   uint32_t T, r_ties, gt_before, eq_before;
   const uint32_t n_c = n_cand;

@@ -106,11 +106,12 @@ def run_path(dw: DeviceWorkload, emit_p: bool | None = None):
     out = torch.empty(wl.B, wl.Lq, wl.H, wl.d_v, dtype=torch.bfloat16, device=dev)
     lse = torch.empty(wl.B, wl.Lq, wl.H, dtype=torch.float32, device=dev)
     p_sel = torch.empty(wl.B, wl.Lq, wl.k, dtype=torch.float32, device=dev) if emit_p else None
-    ws_bytes = max(dsa.dsa_workspace_bytes(dsa.DSA_OP_SPARSE_MLA_FWD, wl.B, wl.Lq, wl.Lk, wl.k, wl.H),
-                   dsa.dsa_workspace_bytes(dsa.DSA_OP_INDEXER_TOPK, wl.B, wl.Lq, wl.Lk, wl.k, 0))
+    ws_bytes = dsa.dsa_workspace_bytes(dsa.DSA_OP_SPARSE_MLA_FWD, wl.B, wl.Lq, wl.Lk, wl.k, wl.H)
     ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
     if wl.Lq == 1:  # decode: the fused indexer -> top-k entry point, as the bench runs it
-        dsa.dsa_indexer_topk(dw.qI, dw.kI, dw.w, scores, idx, ws)
+        ws_ix = torch.zeros(max(16, dsa.dsa_workspace_bytes(dsa.DSA_OP_INDEXER_TOPK, wl.B, 1, wl.Lk, wl.k, 0)),
+                            dtype=torch.uint8, device=dev)  # zero-filled once
+        dsa.dsa_indexer_topk(dw.qI, dw.kI, dw.w, scores, idx, ws_ix)
     else:
         dsa.dsa_indexer(dw.qI, dw.kI, dw.w, scores)
         dsa.dsa_topk(scores, idx)

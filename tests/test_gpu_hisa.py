@@ -28,7 +28,7 @@ def _run(dsa, wl, dw, block, r):
     dsa.dsa_hisa_block_sums(dw.kI, block, sums)
     idx = torch.full((B, 1, k), -7, dtype=torch.int32, device="cuda")
     blocks = torch.full((B, 1, r), -7, dtype=torch.int32, device="cuda")
-    ws = torch.empty(dsa.dsa_hisa_workspace_bytes(B, Lk, block, r, k), dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(dsa.dsa_hisa_workspace_bytes(B, Lk, block, r, k), dtype=torch.uint8, device="cuda")
     dsa.dsa_hisa_topk(dw.qI, dw.kI, dw.w, sums, block, r, idx, blocks, ws)
     assert dsa.dsa_last_device_status() == 0
     return sums.cpu().numpy(), idx.cpu().numpy(), blocks.cpu().numpy()

@@ -67,10 +67,11 @@ def test_paged_decode_matches_the_oracle(dsa, B, max_len, P, k):
     tbl, sl = dev(table), dev(lens)
     scores = torch.full((B, 1, max_len), float("nan"), device="cuda")
     idx = torch.full((B, 1, k), -7, dtype=torch.int32, device="cuda")
-    ws = torch.empty(max(dsa.dsa_workspace_bytes(dsa.DSA_OP_INDEXER_TOPK, B, 1, max_len, k, 0),
-                         dsa.dsa_workspace_bytes(dsa.DSA_OP_SPARSE_MLA_FWD, B, 1, max_len, k, 128)),
+    ws_ix = torch.zeros(dsa.dsa_workspace_bytes(dsa.DSA_OP_INDEXER_TOPK, B, 1, max_len, k, 0), dtype=torch.uint8,
+                        device="cuda")
+    ws = torch.empty(max(16, dsa.dsa_workspace_bytes(dsa.DSA_OP_SPARSE_MLA_FWD, B, 1, max_len, k, 128)),
                      dtype=torch.uint8, device="cuda")
-    dsa.dsa_indexer_topk_paged(qI_t, kI_pages, w_t, tbl, sl, scores, idx, ws)
+    dsa.dsa_indexer_topk_paged(qI_t, kI_pages, w_t, tbl, sl, scores, idx, ws_ix)
     out = torch.empty(B, 1, 128, 512, dtype=torch.bfloat16, device="cuda")
     lse = torch.empty(B, 1, 128, device="cuda")
     dsa.dsa_sparse_mla_fwd_paged(q_t, kv_pages, idx, tbl, sl, max_len, wl.scale, out, lse, ws)
@@ -99,11 +100,12 @@ def test_paged_full_rows_equal_the_contiguous_path(dsa):
     lens = torch.full((B,), L, dtype=torch.int32, device="cuda")
     s1, s2 = (torch.empty(B, 1, L, device="cuda") for _ in range(2))
     i1, i2 = (torch.empty(B, 1, k, dtype=torch.int32, device="cuda") for _ in range(2))
-    ws = torch.empty(max(dsa.dsa_workspace_bytes(dsa.DSA_OP_INDEXER_TOPK, B, 1, L, k, 0),
-                         dsa.dsa_workspace_bytes(dsa.DSA_OP_SPARSE_MLA_FWD, B, 1, L, k, 128)),
+    ws_ix = torch.zeros(dsa.dsa_workspace_bytes(dsa.DSA_OP_INDEXER_TOPK, B, 1, L, k, 0), dtype=torch.uint8,
+                        device="cuda")
+    ws = torch.empty(max(16, dsa.dsa_workspace_bytes(dsa.DSA_OP_SPARSE_MLA_FWD, B, 1, L, k, 128)),
                      dtype=torch.uint8, device="cuda")
-    dsa.dsa_indexer_topk_paged(dw.qI, dw.kI.reshape(B * L // P, P, 128), dw.w, table, lens, s1, i1, ws)
-    dsa.dsa_indexer_topk(dw.qI, dw.kI, dw.w, s2, i2, ws)
+    dsa.dsa_indexer_topk_paged(dw.qI, dw.kI.reshape(B * L // P, P, 128), dw.w, table, lens, s1, i1, ws_ix)
+    dsa.dsa_indexer_topk(dw.qI, dw.kI, dw.w, s2, i2, ws_ix)
     o1, o2 = (torch.empty(B, 1, 128, 512, dtype=torch.bfloat16, device="cuda") for _ in range(2))
     dsa.dsa_sparse_mla_fwd_paged(dw.q, dw.kv.reshape(B * L // P, P, 576), i1, table, lens, L, wl.scale, o1, None, ws)
     dsa.dsa_sparse_mla_fwd(dw.q, dw.kv, i2, wl.scale, o2, None, None, ws)

@@ -248,10 +248,12 @@ def test_fused_indexer_topk_matches_the_two_calls_and_the_oracle(dsa, H_I, B, Lk
     s2 = torch.full((B, 1, Lk), float("nan"), device="cuda")
     i1 = torch.full((B, 1, k), -7, dtype=torch.int32, device="cuda")
     i2 = torch.full((B, 1, k), -7, dtype=torch.int32, device="cuda")
-    ws = torch.full((dsa.dsa_workspace_bytes(dsa.DSA_OP_INDEXER_TOPK, B, 1, Lk, k, 0),), 0xAB,
-                    dtype=torch.uint8, device="cuda")  # garbage: the call clears what it uses
-    for _ in range(2):  # twice: the histograms start from zero on every call
+    ws = torch.zeros(dsa.dsa_workspace_bytes(dsa.DSA_OP_INDEXER_TOPK, B, 1, Lk, k, 0), dtype=torch.uint8,
+                     device="cuda")  # zero-filled once
+    for _ in range(3):  # the call leaves the histograms cleared for the next one
         dsa.dsa_indexer_topk(dw.qI, dw.kI, dw.w, s1, i1, ws)
+    torch.cuda.synchronize()
+    assert int(ws.count_nonzero()) == 0
     dsa.dsa_indexer(dw.qI, dw.kI, dw.w, s2)
     dsa.dsa_topk(s2, i2)
     assert dsa.dsa_last_device_status() == 0
