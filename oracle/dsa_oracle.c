@@ -19,6 +19,9 @@
  *   - dense warm-up loss L^I = sum_t KL(p[t,:] || Softmax(I[t,:])) over every s <= t, with p
  *     the dense main attention summed over heads and L1-normalised, "DSA Continued
  *     Pre-Training" page, Stage 1, and the analysis page eq. (3)
+ *   - masked MHA for short prefill: MLA's MHA mode (per-head decompressed keys and values) with
+ *     every position outside S_t masked, which gives DSA's attention (V3.2-Exp page, sec. 3,
+ *     inference costs; the analysis page's MHA/MQA-mode paragraph, Fig. 7)
  *   - HISA's two-stage retrieval: blocks scored by a block representative, the best blocks'
  *     tokens scored exactly, top-k among them (analysis page, sec. 5.3, eq. (24)-(25) and the
  *     block-mean paragraph)
@@ -247,6 +250,41 @@ double ref_dense_kl_row(const double* scores_row, int t, const double* p) {
     kl += p[s] * (log(p[s]) - (scores_row[s] - log_z));
   }
   return kl;
+}
+
+/* ---- f4: masked MHA (MLA's MHA mode restricted to S_t) ------------------------------------ */
+/* For each head h: z_s = scale * <q[h,:], k[s,h,:]> over the selected positions s of idx (-1 =
+ * empty slot), P = softmax(z), out[h,:] = sum_s P_s v[s,h,:], lse[h] = ln sum_s exp(z_s); a head
+ * with no selected position gets out = 0, lse = -inf.  Real (fp64) inputs: q [H][dqk],
+ * k_seq [L][H][dqk], v_seq [L][H][dv]. */
+void ref_masked_mha_row(const double* q_row, const double* k_seq, const double* v_seq, const int32_t* idx, int k,
+                        int H, int dqk, int dv, double scale, double* out, double* lse) {
+  double* z = (double*)malloc(sizeof(double) * (size_t)(k > 0 ? k : 1));
+  for (int h = 0; h < H; ++h) {
+    double m = -INFINITY;
+    for (int i = 0; i < k; ++i) {
+      if (idx[i] < 0) continue;
+      double dot = 0.0;
+      for (int d = 0; d < dqk; ++d) dot += q_row[h * dqk + d] * k_seq[((int64_t)idx[i] * H + h) * dqk + d];
+      z[i] = scale * dot;
+      if (z[i] > m) m = z[i];
+    }
+    for (int e = 0; e < dv; ++e) out[h * dv + e] = 0.0;
+    if (m == -INFINITY) {
+      lse[h] = -INFINITY;
+      continue;
+    }
+    double denom = 0.0;
+    for (int i = 0; i < k; ++i)
+      if (idx[i] >= 0) denom += exp(z[i] - m);
+    for (int i = 0; i < k; ++i) {
+      if (idx[i] < 0) continue;
+      double p = exp(z[i] - m) / denom;
+      for (int e = 0; e < dv; ++e) out[h * dv + e] += p * v_seq[((int64_t)idx[i] * H + h) * dv + e];
+    }
+    lse[h] = m + log(denom);
+  }
+  free(z);
 }
 
 /* ---- f4: HISA, block -> token retrieval (analysis page, sec. 5.3) ----------------------- */

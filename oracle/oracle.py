@@ -49,6 +49,7 @@ def _load():
         lib.ref_dense_p_row.argtypes = [vp, vp, i32, i32, i32, f64, vp]
         lib.ref_dense_kl_row.argtypes = [vp, i32, vp]
         lib.ref_dense_kl_row.restype = f64
+        lib.ref_masked_mha_row.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, f64, vp, vp]
         lib.ref_block_mean.argtypes = [vp, i32, i32, i32, vp]
         lib.ref_block_score.argtypes = [vp, vp, vp, i32, i32]
         lib.ref_block_score.restype = f64
@@ -156,6 +157,22 @@ def dense_kl_row(scores_row, t: int, p) -> float:
     scores_row, sp = _c(scores_row, np.float64)
     p, pp = _c(p, np.float64)
     return _load().ref_dense_kl_row(sp, t, pp)
+
+
+def masked_mha_row(q_row, k_seq, v_seq, idx, scale: float):
+    """MHA-mode attention of one query restricted to the positions of idx: q_row [H, dqk],
+    k_seq [L, H, dqk], v_seq [L, H, dv] (real values); returns (out [H, dv], lse [H])."""
+    q_row, qp = _c(q_row, np.float64)
+    k_seq, kp = _c(k_seq, np.float64)
+    v_seq, vp_ = _c(v_seq, np.float64)
+    idx, ip = _c(idx, np.int32)
+    H, dqk = q_row.shape
+    dv = v_seq.shape[2]
+    out = np.empty((H, dv))
+    lse = np.empty(H)
+    _load().ref_masked_mha_row(qp, kp, vp_, ip, idx.shape[0], H, dqk, dv, float(scale), out.ctypes.data,
+                               lse.ctypes.data)
+    return out, lse
 
 
 def block_mean(k_seq, s0: int, n: int) -> np.ndarray:
