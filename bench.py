@@ -542,6 +542,114 @@ def measure(shard, device, steps, warmup, world, peaks, e2e=True):
             "gpu_launches": step.launches_per_step * steps}
 
 
+def time_calls(fn, steps, warmup, flush):
+    """Median device time (ms) of fn() over `steps` calls after `warmup`, L2 flushed before each,
+    CUDA events on the launching stream; also the clocks sampled meanwhile."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    ts = []
+    with ClockSampler(pci_id(flush.device)) as clk:
+        for i in range(steps):
+            flush.fill_(i & 0xFF)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+    return statistics.median(ts), clk.summary()
+
+
+def variant_blocks(device, peaks, steps, warmup):
+    """The NEXT rows, each timed on its own: the indexer-loss backward on the sparse-stage
+    workload's inputs, HISA's decode selection and a paged decode with ragged context lengths."""
+    import sparse_attention_tcgen05_b200 as dsa
+
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    out = {}
+    bf16 = peaks["bf16_tflops"]
+
+    # ---- indexer-loss backward (dq, dw, dk) after one sparse-stage forward
+    wl = dsa_inputs.WORKLOADS["indexer_kl_16k"]
+    st = Step(make_shard(wl, 0, 1, "weak"), device, keep_host=False)
+    st.run()
+    rows, Lk, k = wl.rows, wl.Lk, wl.k
+    dq = torch.empty(wl.B, wl.Lq, wl.H_I, wl.d_I, device=device)
+    dwt = torch.empty(wl.B, wl.Lq, wl.H_I, device=device)
+    dk = torch.empty(wl.B, Lk, wl.d_I, device=device)
+    d = st.d
+    fn = lambda: dsa.dsa_indexer_bwd(d["qI"], d["kI"], d["w"], st.scores, st.idx, st.p, dq, dwt, dk)
+    ms, clk = time_calls(fn, steps, warmup, flush)
+    nsel = float(np.minimum(k, np.arange(wl.Lq) + 1).sum()) * wl.B
+    macs8 = nsel * wl.H_I * wl.d_I                 # a = q . k recomputed (FP8)
+    macs16 = 4 * nsel * wl.H_I * wl.d_I            # dq and dk, each on two fp16 parts
+    tc_us = (2 * macs8 / (FP8_OVER_BF16 * bf16 * 1e12) + 2 * macs16 / (bf16 * 1e12)) * 1e6
+    byts = rows * wl.H_I * (wl.d_I + 4) + Lk * wl.d_I + rows * k * 12 + rows * wl.H_I * (wl.d_I + 1) * 4 + \
+        Lk * wl.d_I * 4 * 2
+    hbm_us = byts / (peaks["hbm_gbs"] * 1e9) * 1e6
+    out["indexer_bwd_16k"] = {
+        "what": "dsa_indexer_bwd on indexer_kl_16k's own scores, idx and p (dq, dw, dk)", "ms": round(ms, 4),
+        "roofline_us": round(max(tc_us, hbm_us), 1), "bound": "tensor" if tc_us > hbm_us else "hbm",
+        "frac": round(max(tc_us, hbm_us) / (ms * 1e3), 4),
+        "tflops": round(2 * (macs8 + macs16) / (ms * 1e-3) / 1e12, 1), "clocks": clk}
+    del st, dq, dwt, dk
+    torch.cuda.empty_cache()
+
+    # ---- HISA and paged decode on the 128K decode workload
+    wl = dsa_inputs.WORKLOADS["decode_128k"]
+    st = Step(make_shard(wl, 0, 1, "weak"), device, keep_host=False)
+    d = st.d
+    B, L, k = wl.B, wl.Lk, wl.k
+    st.run()  # the DSA selection, for the recall of HISA's
+    dsa_idx = st.idx.clone()
+    block, r = 64, 64
+    sums = torch.empty(B, L // block, wl.d_I, device=device)
+    dsa.dsa_hisa_block_sums(d["kI"], block, sums)  # cache summary: once, outside the timed steps
+    hidx = torch.empty(B, 1, k, dtype=torch.int32, device=device)
+    hws = torch.zeros(dsa.dsa_hisa_workspace_bytes(B, L, block, r, k), dtype=torch.uint8, device=device)
+
+    def hisa_step():
+        dsa.dsa_hisa_topk(d["qI"], d["kI"], d["w"], sums, block, r, hidx, None, hws)
+        dsa.dsa_sparse_mla_fwd(d["q"], d["kv"], hidx, wl.scale, st.out, st.lse, None, st.ws)
+
+    ms, clk = time_calls(hisa_step, steps, warmup, flush)
+    ms_sel, _ = time_calls(lambda: dsa.dsa_hisa_topk(d["qI"], d["kI"], d["w"], sums, block, r, hidx, None, hws),
+                           steps, warmup, flush)
+    a, b = dsa_idx.view(B, k), hidx.view(B, k)
+    recall = float(np.mean([np.intersect1d(a[i].cpu().numpy(), b[i].cpu().numpy()).size / k for i in range(B)]))
+    out["decode_128k_hisa"] = {
+        "what": f"HISA selection (blocks of {block}, r = {r}: {r * block} candidate keys) + sparse MLA, "
+                "block sums computed once outside the steps", "ms_per_step": round(ms, 4),
+        "selection_ms": round(ms_sel, 4), "value": B / (ms * 1e-3), "unit": "query-tokens/s",
+        "recall_vs_dsa": round(recall, 4), "clocks": clk}
+
+    # paged cache: pages of 64 keys in a shuffled pool, context lengths uniform in [L/2, L]
+    P = 64
+    g = torch.Generator().manual_seed(0xD5A0 + 77)
+    table = torch.randperm(B * (L // P), generator=g).to(torch.int32).reshape(B, L // P).to(device)
+    lens = torch.randint(L // 2, L + 1, (B,), generator=g, dtype=torch.int32).to(device)
+    kp = d["kI"].reshape(B * L // P, P, wl.d_I)
+    kvp = d["kv"].reshape(B * L // P, P, wl.d_qk)
+    pws = torch.zeros(dsa.dsa_workspace_bytes(dsa.DSA_OP_INDEXER_TOPK, B, 1, L, k, 0), dtype=torch.uint8,
+                      device=device)
+
+    def paged_step():
+        dsa.dsa_indexer_topk_paged(d["qI"], kp, d["w"], table, lens, st.scores, st.idx, pws)
+        dsa.dsa_sparse_mla_fwd_paged(d["q"], kvp, st.idx, table, lens, L, wl.scale, st.out, st.lse, st.ws)
+
+    ms, clk = time_calls(paged_step, steps, warmup, flush)
+    tot = float(lens.sum().item())
+    byts = tot * wl.d_I + B * k * wl.d_qk * 2 + B * wl.H * (wl.d_qk + wl.d_v) * 2
+    out["decode_128k_paged"] = {
+        "what": f"paged decode, pages of {P} keys in a shuffled pool, seq_lens uniform in [{L // 2}, {L}] "
+                f"(mean {tot / B:.0f})", "ms_per_step": round(ms, 4), "value": B / (ms * 1e-3),
+        "unit": "query-tokens/s", "hbm_roofline_us": round(byts / (peaks["hbm_gbs"] * 1e9) * 1e6, 1),
+        "clocks": clk}
+    assert dsa.dsa_last_device_status() == 0
+    return out
+
+
 def workload_config(wl, world=1, scaling="weak", shard=None):
     cfg = {"workload": wl.name, "B": wl.B, "Lq": wl.Lq, "Lk": wl.Lk, "H_I": wl.H_I,
            "d_I": wl.d_I, "k": wl.k, "H": wl.H, "d_qk": wl.d_qk, "d_v": wl.d_v,
@@ -598,6 +706,8 @@ def gpu_arm(args, rank, world, device):
         line["workloads"] = extra
         line["gpu_launches"] += sum(r["gpu_launches"] for r in extra.values()) + \
             line.get("north_star", {}).get("gpu_launches", 0)
+        torch.cuda.empty_cache()
+        line["variants"] = variant_blocks(device, peaks, args.extra_steps, 3)
     return line
 
 

@@ -59,7 +59,8 @@ enum {
   DSA_OP_INDEXER_KL = 3,
   DSA_OP_DENSE_MLA_FWD = 4,
   DSA_OP_INDEXER_KL_DENSE = 5,
-  DSA_OP_INDEXER_TOPK = 6
+  DSA_OP_INDEXER_TOPK = 6,
+  DSA_OP_MASKED_MHA = 7
 };
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -160,6 +161,26 @@ dsa_status dsa_sparse_mla_fwd_paged(const void* q_bf16, const void* kv_pages, co
                                     int max_len, int num_pages, int page_size, int H, int d_qk,
                                     int d_v, int k, float scale, void* out_bf16, float* lse, void* ws,
                                     size_t ws_bytes, dsa_stream_t stream);
+
+/*
+ * Masked MHA for short prefill ("DeepSeek-V3.2-Exp" page, sec. 3, inference costs: for short
+ * prefills DSA is simulated with MLA's MHA mode and a mask; "DeepSeek-V3.2" analysis page,
+ * sec. 1.1, the MHA/MQA-mode paragraph and Fig. 7).  In MHA mode every head h has its own
+ * decompressed keys and values; query t of head h attends only to the positions of its top-k
+ * set S_t (idx, -1 = empty slot; a position is used only if it is also <= t):
+ *   z_s = scale * <q[b,t,h,:], k[b,s,h,:]>,  P = softmax over s in S_t, s <= t
+ *   out[b,t,h,:] = sum_s P_s v[b,s,h,:],  lse[b,t,h] = ln sum_s exp(z_s)
+ * This equals DSA's MQA-mode attention over S_t once the decompression is absorbed.
+ *   q_bf16, k_bf16 [B, L, H, 192] bf16 (128 + 64 rope dims), v_bf16 [B, L, H, 128] bf16,
+ *   idx [B, L, k] int32, out_bf16 [B, L, H, 128] bf16, lse [B, L, H] fp32 (nullable)
+ *   ws: dsa_workspace_bytes(DSA_OP_MASKED_MHA, B, L, L, k, H) bytes (the selection bitmap)
+ * Causal prefill only (every query of the sequence, t = 0 .. L-1).  bf16 tensor-core products,
+ * fp32 softmax and accumulation.  Supported: d_qk = 192, d_v = 128, L <= 65536.
+ */
+dsa_status dsa_masked_mha_fwd(const void* q_bf16, const void* k_bf16, const void* v_bf16,
+                              const int32_t* idx, int B, int L, int H, int d_qk, int d_v, int k,
+                              float scale, void* out_bf16, float* lse, void* ws, size_t ws_bytes,
+                              dsa_stream_t stream);
 
 /*
  * HISA, block -> token retrieval for decode ("DeepSeek-V3.2" analysis page, sec. 5.3: a coarse

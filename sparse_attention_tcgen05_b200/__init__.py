@@ -21,18 +21,19 @@ __all__ = [
     "dsa_last_device_status", "dsa_set_wait_limit_ns", "dsa_selftest_wait", "dsa_dense_mla_fwd",
     "dsa_indexer_kl_dense", "dsa_indexer_topk", "dsa_indexer_bwd", "dsa_indexer_topk_paged",
     "dsa_sparse_mla_fwd_paged", "dsa_hisa_workspace_bytes", "dsa_hisa_block_sums", "dsa_hisa_topk",
+    "dsa_masked_mha_fwd",
     "DSA_OP_INDEXER", "DSA_OP_TOPK", "DSA_OP_SPARSE_MLA_FWD", "DSA_OP_INDEXER_KL",
-    "DSA_OP_DENSE_MLA_FWD", "DSA_OP_INDEXER_KL_DENSE", "DSA_OP_INDEXER_TOPK", "EXPORTED",
+    "DSA_OP_DENSE_MLA_FWD", "DSA_OP_INDEXER_KL_DENSE", "DSA_OP_INDEXER_TOPK", "DSA_OP_MASKED_MHA", "EXPORTED",
 ]
 
 DSA_OP_INDEXER, DSA_OP_TOPK, DSA_OP_SPARSE_MLA_FWD, DSA_OP_INDEXER_KL = 0, 1, 2, 3
-DSA_OP_DENSE_MLA_FWD, DSA_OP_INDEXER_KL_DENSE, DSA_OP_INDEXER_TOPK = 4, 5, 6
+DSA_OP_DENSE_MLA_FWD, DSA_OP_INDEXER_KL_DENSE, DSA_OP_INDEXER_TOPK, DSA_OP_MASKED_MHA = 4, 5, 6, 7
 EXPORTED = ("dsa_status_str", "dsa_version", "dsa_workspace_bytes", "dsa_indexer", "dsa_topk",
             "dsa_sparse_mla_fwd", "dsa_indexer_kl", "dsa_indexer_kl_noalloc",
             "dsa_last_device_status", "dsa_set_wait_limit_ns", "dsa_selftest_wait",
             "dsa_dense_mla_fwd", "dsa_indexer_kl_dense", "dsa_indexer_topk", "dsa_indexer_bwd",
             "dsa_indexer_topk_paged", "dsa_sparse_mla_fwd_paged", "dsa_hisa_workspace_bytes",
-            "dsa_hisa_block_sums", "dsa_hisa_topk")
+            "dsa_hisa_block_sums", "dsa_hisa_topk", "dsa_masked_mha_fwd")
 
 
 class DsaError(RuntimeError):
@@ -79,11 +80,12 @@ def load(rebuild: bool = False) -> ctypes.CDLL:
         lib.dsa_hisa_workspace_bytes.restype = sz
         lib.dsa_hisa_block_sums.argtypes = [vp, i32, i32, i32, i32, vp, vp]
         lib.dsa_hisa_topk.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, vp, vp, vp, sz, vp]
+        lib.dsa_masked_mha_fwd.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, vp, vp, vp, sz, vp]
         for name in ("dsa_indexer", "dsa_topk", "dsa_sparse_mla_fwd", "dsa_indexer_kl",
                      "dsa_indexer_kl_noalloc", "dsa_last_device_status", "dsa_set_wait_limit_ns",
                      "dsa_selftest_wait", "dsa_dense_mla_fwd", "dsa_indexer_kl_dense", "dsa_indexer_topk",
                      "dsa_indexer_bwd", "dsa_indexer_topk_paged", "dsa_sparse_mla_fwd_paged",
-                     "dsa_hisa_block_sums", "dsa_hisa_topk"):
+                     "dsa_hisa_block_sums", "dsa_hisa_topk", "dsa_masked_mha_fwd"):
             getattr(lib, name).restype = i32
         _lib = lib
     return _lib
@@ -361,6 +363,27 @@ def dsa_hisa_topk(q_fp8: torch.Tensor, k_fp8: torch.Tensor, w: torch.Tensor, sum
     _raise("dsa_hisa_topk",
            load().dsa_hisa_topk(_ptr(q_fp8), _ptr(k_fp8), _ptr(w), _ptr(sums), B, Lk, H_I, d_I, block, r, k,
                                 _ptr(idx), _ptr(blocks), wsp, wsb, _stream(stream)))
+
+
+def dsa_masked_mha_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, idx: torch.Tensor, scale: float,
+                       out: torch.Tensor, lse: torch.Tensor | None = None, ws: torch.Tensor | None = None,
+                       stream=None) -> None:
+    """MHA-mode causal prefill attention of q/k [B,L,H,192], v [B,L,H,128] (bf16) restricted to each
+    query's top-k set idx [B,L,k]; out [B,L,H,128] bf16, optional lse [B,L,H]."""
+    B, L, H, d_qk = q.shape
+    kk = idx.shape[2]
+    d_v = v.shape[3]
+    _check(q, "q", torch.bfloat16, (B, L, H, d_qk))
+    _check(k, "k", torch.bfloat16, (B, L, H, d_qk))
+    _check(v, "v", torch.bfloat16, (B, L, H, d_v))
+    _check(idx, "idx", torch.int32, (B, L, kk))
+    _check(out, "out", torch.bfloat16, (B, L, H, d_v))
+    if lse is not None:
+        _check(lse, "lse", torch.float32, (B, L, H))
+    wsp, wsb = _ws(ws)
+    _raise("dsa_masked_mha_fwd",
+           load().dsa_masked_mha_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(idx), B, L, H, d_qk, d_v, kk, float(scale),
+                                     _ptr(out), _ptr(lse), wsp, wsb, _stream(stream)))
 
 
 def dsa_indexer_kl_noalloc(scores: torch.Tensor, idx: torch.Tensor, p_sel: torch.Tensor,

@@ -16,6 +16,7 @@
 #include "indexer.cuh"
 #include "indexer_bwd.cuh"
 #include "indexer_kl.cuh"
+#include "masked_mha.cuh"
 #include "ptx.cuh"
 #include "sparse_mla.cuh"
 #include "sparse_mla_pair.cuh"
@@ -493,6 +494,8 @@ size_t dsa_workspace_bytes(int op, int B, int Lq, int Lk, int k, int H) {
       return std::max(mla_ws_bytes(static_cast<int>(rows), Lk, H, 512, sms),
                       mla_ws_bytes(static_cast<int>(rows), Lk, H, 64, sms));
     }
+    case DSA_OP_MASKED_MHA:  // the selection bitmap, rows of a multiple of 4 words
+      return static_cast<size_t>(rows) * (((Lk + 127) / 128) * 4) * sizeof(uint32_t);
     case DSA_OP_INDEXER_TOPK:
       // the decode kernels' top-digit histograms (no workspace for other shapes)
       return Lq == 1 ? static_cast<size_t>(rows) * 2048 * sizeof(uint32_t) : 0;
@@ -867,6 +870,60 @@ dsa_status dsa_hisa_topk(const void* q_fp8, const void* k_fp8, const float* w, c
   // 5. candidate slots -> positions
   return launch(dsa::hisa::slots_to_positions_kernel, static_cast<unsigned>(B), 256u, 0, st, 1,
                 static_cast<const int32_t*>(cidx), static_cast<const int32_t*>(bidx), r, block, k, idx);
+}
+
+dsa_status dsa_masked_mha_fwd(const void* q_bf16, const void* k_bf16, const void* v_bf16, const int32_t* idx, int B,
+                              int L, int H, int d_qk, int d_v, int k, float scale, void* out_bf16, float* lse,
+                              void* ws, size_t ws_bytes, dsa_stream_t stream) {
+  if (!q_bf16 || !k_bf16 || !v_bf16 || !idx || !out_bf16 || !ws) return DSA_ERR_INVALID_ARG;
+  if (B <= 0 || L <= 0 || H <= 0 || k <= 0) return DSA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q_bf16) || !aligned16(k_bf16) || !aligned16(v_bf16) || !aligned16(idx) || !aligned16(out_bf16) ||
+      (lse && !aligned16(lse)) || !aligned16(ws))
+    return DSA_ERR_INVALID_ARG;
+  if (d_qk != dsa::mmha::kDQK || d_v != dsa::mmha::kDV || L > 65536) return DSA_ERR_UNSUPPORTED;
+  const int words = ((L + 127) / 128) * 4;
+  const size_t need = static_cast<size_t>(B) * L * words * sizeof(uint32_t);
+  if (ws_bytes < need) return DSA_ERR_INVALID_ARG;
+  const long n_qt = (L + dsa::mmha::kBM - 1) / dsa::mmha::kBM;
+  if (static_cast<long>(B) * L * H >= INT32_MAX || static_cast<long>(B) * H * n_qt >= INT32_MAX ||
+      static_cast<long>(B) * L >= INT32_MAX)
+    return DSA_ERR_UNSUPPORTED;
+  DeviceInfo dev;
+  const dsa_status ds = current_device(dev);
+  if (ds != DSA_OK) return ds;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t* sel = static_cast<uint32_t*>(ws);
+  if (cudaFuncSetAttribute(dsa::mmha::build_selection_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           words * 4) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  dsa_status s = launch(dsa::mmha::build_selection_kernel, static_cast<unsigned>(B * L), 256u,
+                        static_cast<size_t>(words) * 4, st, 1, idx, L, k, words, sel);
+  if (s != DSA_OK) return s;
+  // q, k: [B * L rows, H * 192 cols]; v: [B * L rows, H * 128 cols]; boxes of 64 cols x 128 rows
+  CUtensorMap tm_q, tm_k, tm_v;
+  const uint64_t rows = static_cast<uint64_t>(B) * L;
+  if (!encode_2d(&tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q_bf16, static_cast<uint64_t>(H) * d_qk, rows,
+                 static_cast<uint64_t>(H) * d_qk * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_2d(&tm_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, k_bf16, static_cast<uint64_t>(H) * d_qk, rows,
+                 static_cast<uint64_t>(H) * d_qk * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_2d(&tm_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, v_bf16, static_cast<uint64_t>(H) * d_v, rows,
+                 static_cast<uint64_t>(H) * d_v * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+    return DSA_ERR_CUDA;
+  dsa::mmha::Params p{};
+  p.sel = sel;
+  p.out = static_cast<__nv_bfloat16*>(out_bf16);
+  p.lse = lse;
+  p.B = B;
+  p.L = L;
+  p.H = H;
+  p.words = words;
+  p.scale_log2 = scale * dsa::mla::kLog2e;
+  auto kern = dsa::mmha::masked_mha_kernel;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dsa::mmha::kSmemBytes) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  return launch(kern, static_cast<unsigned>(B * H * n_qt), dsa::mmha::kThreads, dsa::mmha::kSmemBytes, st, 1, tm_q,
+                tm_k, tm_v, p);
 }
 
 dsa_status dsa_set_wait_limit_ns(uint64_t ns) {
