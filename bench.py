@@ -646,6 +646,38 @@ def variant_blocks(device, peaks, steps, warmup):
                 f"(mean {tot / B:.0f})", "ms_per_step": round(ms, 4), "value": B / (ms * 1e-3),
         "unit": "query-tokens/s", "hbm_roofline_us": round(byts / (peaks["hbm_gbs"] * 1e9) * 1e6, 1),
         "clocks": clk}
+    del st, kp, kvp
+    torch.cuda.empty_cache()
+
+    # ---- masked MHA (MHA mode, per-head keys and values) on a 4K prefill's own top-k sets,
+    # against the MQA-mode sparse kernel on the same sets
+    wl = dsa_inputs.WORKLOADS["prefill_1x4k"]
+    st = Step(make_shard(wl, 0, 1, "weak"), device, keep_host=False)
+    st.run()
+    L, H, k = wl.Lk, wl.H, wl.k
+    gen = lambda tid, shape: torch.from_numpy(
+        dsa_inputs.normal_bf16_bits(wl.seed, tid, int(np.prod(shape))).view(np.int16).reshape(shape)).view(
+        torch.bfloat16).to(device)
+    qm, km, vm = gen(11, (1, L, H, 192)), gen(12, (1, L, H, 192)), gen(13, (1, L, H, 128))
+    om = torch.empty(1, L, H, 128, dtype=torch.bfloat16, device=device)
+    lm = torch.empty(1, L, H, device=device)
+    mws = torch.empty(dsa.dsa_workspace_bytes(dsa.DSA_OP_MASKED_MHA, 1, L, L, k, H), dtype=torch.uint8,
+                      device=device)
+    ms_mha, clk = time_calls(lambda: dsa.dsa_masked_mha_fwd(qm, km, vm, st.idx, 1 / np.sqrt(192.0), om, lm, mws),
+                             steps, warmup, flush)
+    d = st.d
+    ms_mqa, _ = time_calls(lambda: dsa.dsa_sparse_mla_fwd(d["q"], d["kv"], st.idx, wl.scale, st.out, st.lse, None,
+                                                          st.ws), steps, warmup, flush)
+    pairs = L * (L + 1) / 2
+    nsel = float(np.minimum(k, np.arange(L) + 1).sum())
+    fl_mha = 2 * pairs * H * (192 + 128)   # every causal (t, s) of the tiles the kernel visits
+    fl_mqa = 2 * nsel * H * (576 + 512)
+    out["prefill_4k_masked_mha"] = {
+        "what": "masked MHA (MHA mode: 192-d keys, 128-d values per head) vs the MQA-mode sparse kernel, "
+                "prefill_1x4k's own top-k sets", "masked_mha_ms": round(ms_mha, 4), "mqa_sparse_ms": round(ms_mqa, 4),
+        "masked_mha_tflops": round(fl_mha / (ms_mha * 1e-3) / 1e12, 1),
+        "masked_mha_tensor_frac": round(fl_mha / (ms_mha * 1e-3) / 1e12 / bf16, 4),
+        "mqa_sparse_tflops": round(fl_mqa / (ms_mqa * 1e-3) / 1e12, 1), "clocks": clk}
     assert dsa.dsa_last_device_status() == 0
     return out
 
