@@ -74,8 +74,8 @@ struct Cfg {
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kOffQ + 2 * ((kQBytes + 1023) / 1024) * 1024;
   static constexpr int kOffW = kOffK + kStages * kKBytes;
-  static constexpr int kOffHist = kOffW + 2 * N * 4;                 // decode: [2048] digit counts
-  static constexpr int kOffBar = kOffHist + (G == 1 ? 2048 * 4 : 0);
+  static constexpr int kOffHist = kOffW + 2 * N * 4;                 // decode: [2 groups][2048] digit counts
+  static constexpr int kOffBar = kOffHist + (G == 1 ? 2 * 2048 * 4 : 0);
   static constexpr int kNumBars = 2 * kStages + 8;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
@@ -276,8 +276,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     int gt = 0;  // tiles with an MMA seen so far, over all items (both groups count every one)
     int it = 0;
     const bool count = (G == 1) && p.hist != nullptr;
+    uint32_t* gHist = sHist + wg * 2048;  // this warpgroup's counts (decode: the groups take turns by tile)
     if (count)
-      for (int x = e; x < 2048; x += 256) sHist[x] = 0u;  // ordered by the item's first barrier
+      for (int x = e & 127; x < 2048; x += 128) gHist[x] = 0u;  // ordered by the item's first barrier
     for (int u = blockIdx.x; u < p.n_items; u += gridDim.x, ++it) {
       int b, qg, kc, kt0, kt1, n_comp;
       decode_item(p, u, b, qg, kc);
@@ -336,18 +337,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int t = query_pos(p, b, i0);
             const uint32_t bin = (s < p.Lk && s <= t) ? (ordered_key(acc[0]) >> 21) : 0xFFFFFFFFu;
             const uint32_t peers = __match_any_sync(0xFFFFFFFFu, bin);
-            if (bin != 0xFFFFFFFFu && lane == __ffs(peers) - 1) atomicAdd(&sHist[bin], __popc(peers));
+            if (bin != 0xFFFFFFFFu && lane == __ffs(peers) - 1) atomicAdd(&gHist[bin], __popc(peers));
           }
         }
       }
-      if (count) {  // this item's counts into the row's histogram; the next item starts from zero
-        named_bar_sync(2, 256);
+      if (count) {  // this group's counts of the item into the row's histogram; the next item starts
+                    // from zero (the groups flush independently, each behind its own barrier)
+        named_bar_sync(2 + wg, 128);
         uint32_t* gh = p.hist + (row_base + i0) * 2048;
-        for (int x = e; x < 2048; x += 256) {
-          const uint32_t v = sHist[x];
+        for (int x = e & 127; x < 2048; x += 128) {
+          const uint32_t v = gHist[x];
           if (v) {
             atomicAdd(gh + x, v);
-            sHist[x] = 0u;
+            gHist[x] = 0u;
           }
         }
       }

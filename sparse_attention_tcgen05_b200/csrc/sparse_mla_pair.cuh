@@ -199,6 +199,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_proxy_async_smem();
   }
   pdl_launch_dependents();
+  if (threadIdx.x == kMmaWarp * 32) {
+    // this CTA's Q slice into L2 while the previous kernel of the stream finishes (a prefetch
+    // only warms the cache; the loads below come after the dependency wait)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) tma_prefetch_2d(&tm_q_main, static_cast<int>(rank) * kDvCta + i * 64, row * p.H);
+    tma_prefetch_2d(&tm_q_rope, kDV + static_cast<int>(rank) * kRopeCta, row * p.H);
+  }
   if (warp == kMmaWarp) tmem_alloc(tmem_slot, kTmemCols);
   tc_fence_before();
   // the peer's barriers must be initialised before any remote store completes on them

@@ -228,7 +228,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int row = blockIdx.x / C;
   const uint32_t rank = (C > 1) ? cluster_ctarank() : 0u;
   const int i = row % Lq;
-  // decode rows of a paged cache (Lq == 1) see their own context length, clamped to [0, Lk]
+  // decode rows of a paged cache (Lq == 1) see their own context length, clamped to [0, Lk]; the
+  // lengths may come from an earlier kernel of the stream, so wait for it first
+  if (seq_lens) pdl_wait();
   const int t = seq_lens ? min(max(__ldg(seq_lens + row / Lq), 0), Lk) - 1 : i + Lk - Lq;
   const int n = t + 1;  // candidates s in [0, n)
   int32_t* out = idx + static_cast<size_t>(row) * k;

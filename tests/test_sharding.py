@@ -86,3 +86,37 @@ def test_helpers_are_identity_on_one_process():
     x = torch.tensor([2.5])
     assert sharding.sum_over_ranks(x) is x and x.item() == 2.5
     assert sharding.max_over_ranks(3.0) == 3.0
+
+
+@pytest.mark.parametrize("Lq,Lk,world", [(160, 160, 3), (120, 250, 2)])
+def test_causal_shard_calls_reproduce_the_whole_sequence_rows(Lq, Lk, world):
+    # a rank calls the path on its rows with Lq' = stop - start and Lk' = stop + (Lk - Lq) over the
+    # key prefix [0, Lk'): each of its rows must get the whole sequence's scores, top-k set and
+    # attention output (the oracle run both ways)
+    import dsa_inputs
+    H_I, d_I, k, H, d_qk, d_v = 2, 16, 24, 2, 40, 32
+    seed = 0x5A4D + Lq
+    qI = dsa_inputs.e4m3_small_int(seed, 1, Lq * H_I * d_I).reshape(Lq, H_I, d_I)
+    kI = dsa_inputs.e4m3_small_int(seed, 2, Lk * d_I).reshape(Lk, d_I)
+    w = (dsa_inputs.uniform_int(seed, 3, Lq * H_I, -8, 8) / 8.0).astype(np.float32).reshape(Lq, H_I)
+    q = dsa_inputs.normal_bf16_bits(seed, 4, Lq * H * d_qk).reshape(Lq, H, d_qk)
+    kv = dsa_inputs.normal_bf16_bits(seed, 5, Lk * d_qk).reshape(Lk, d_qk)
+    scale = 1 / np.sqrt(d_qk)
+    for rank in range(world):
+        start, stop = sharding.shard_causal_rows(Lq, Lk, k, rank, world, mla_weight=sharding.MLA_WEIGHT)
+        Lq_loc, Lk_loc = stop - start, stop + (Lk - Lq)
+        for i in (0, Lq_loc // 2, Lq_loc - 1):
+            g = start + i
+            t_full, t_loc = g + Lk - Lq, i + Lk_loc - Lq_loc
+            assert t_loc == t_full
+            s_full = ref.indexer_row(qI[g], kI, w[g], t_full)
+            s_loc = ref.indexer_row(qI[g], kI[:Lk_loc], w[g], t_loc)
+            np.testing.assert_array_equal(s_loc[: t_loc + 1], s_full[: t_full + 1])
+            idx_full, n_full = ref.topk_row(s_full, t_full, k)
+            idx_loc, n_loc = ref.topk_row(s_loc, t_loc, k)
+            np.testing.assert_array_equal(idx_loc, idx_full)
+            assert n_loc == n_full
+            o_full, lse_full, _ = ref.sparse_mla_row(q[g], kv, idx_full, d_v, scale)
+            o_loc, lse_loc, _ = ref.sparse_mla_row(q[g], kv[:Lk_loc], idx_loc, d_v, scale)
+            np.testing.assert_array_equal(o_loc, o_full)
+            np.testing.assert_array_equal(lse_loc, lse_full)
