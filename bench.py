@@ -103,9 +103,6 @@ def algorithmic(wl):
         ml["macs"] += nsel * wl.H * wl.d_qk
         ml["bytes"] += 4 * B * Lq * k
     kl = {"bytes": 4 * nsel + 8 * B * Lq * k, "macs": 0.0}
-    if Lq == 1:  # decode runs the fused indexer -> top-k: one stage, the two stages' work
-        return {"indexer_topk": {"bytes": ix["bytes"] + tk["bytes"], "macs": ix["macs"]}, "sparse_mla": ml,
-                "indexer_kl": kl}
     return {"indexer": ix, "topk": tk, "sparse_mla": ml, "indexer_kl": kl}
 
 
@@ -317,10 +314,6 @@ class Step:
         pk = Lk if wl.dense else wl.k  # the dense target covers every position
         self.p = torch.empty(B, Lq, pk, dtype=torch.float32, device=device) if wl.emit_p else None
         self.loss = torch.empty(1, dtype=torch.float32, device=device)
-        # the fused decode indexer -> top-k keeps its histograms zero-filled between calls: a
-        # buffer of its own, cleared once
-        self.ws_ix = torch.zeros(max(16, dsa.dsa_workspace_bytes(dsa.DSA_OP_INDEXER_TOPK, B, Lq, Lk, wl.k, 0)),
-                                 dtype=torch.uint8, device=device)
         nws = max(dsa.dsa_workspace_bytes(dsa.DSA_OP_SPARSE_MLA_FWD, B, Lq, Lk, wl.k, wl.H),
                   dsa.dsa_workspace_bytes(dsa.DSA_OP_DENSE_MLA_FWD, B, Lq, Lk, 0, wl.H) if wl.dense else 0,
                   dsa.dsa_workspace_bytes(dsa.DSA_OP_INDEXER_KL, B, Lq, Lk, wl.k, 0), 16)
@@ -347,16 +340,6 @@ class Step:
         dsa, d, wl = self.dsa, self.d, self.wl
         if ev:
             ev[0].record()
-        if wl.Lq == 1 and not wl.dense:  # decode: the fused indexer -> top-k (one stage)
-            dsa.dsa_indexer_topk(d["qI"], d["kI"], d["w"], self.scores, self.idx, self.ws_ix)
-            if ev:
-                ev[1].record()
-                ev[2].record()
-            dsa.dsa_sparse_mla_fwd(d["q"], d["kv"], self.idx, wl.scale, self.out, self.lse, self.p, self.ws)
-            if ev:
-                ev[3].record()
-                ev[4].record()
-            return
         dsa.dsa_indexer(d["qI"], d["kI"], d["w"], self.scores)
         if ev:
             ev[1].record()
@@ -473,9 +456,6 @@ def measure(shard, device, steps, warmup, world, peaks, e2e=True):
         stage_ms[attn].append(e[2].elapsed_time(e[3]))
         stage_ms["indexer_kl"].append(e[3].elapsed_time(e[4]))
     if wl.dense:
-        del stage_ms["topk"]
-    if wl.Lq == 1 and not wl.dense:  # the fused decode call: indexer and top-k are one stage
-        stage_ms["indexer_topk"] = stage_ms.pop("indexer")
         del stage_ms["topk"]
     total_ms = max_over_ranks(sum(step_ms), device)  # the slowest rank's time
     ms_per_step = total_ms / steps
@@ -603,6 +583,23 @@ def variant_blocks(device, peaks, steps, warmup):
     B, L, k = wl.B, wl.Lk, wl.k
     st.run()  # the DSA selection, for the recall of HISA's
     dsa_idx = st.idx.clone()
+
+    # the fused indexer -> top-k call (the indexer counts the top-k's first radix digit in its
+    # epilogue) against the two separate calls, each step followed by the sparse MLA
+    ws_ix = torch.zeros(max(16, dsa.dsa_workspace_bytes(dsa.DSA_OP_INDEXER_TOPK, B, 1, L, k, 0)),
+                        dtype=torch.uint8, device=device)
+
+    def fused_step():
+        dsa.dsa_indexer_topk(d["qI"], d["kI"], d["w"], st.scores, st.idx, ws_ix)
+        dsa.dsa_sparse_mla_fwd(d["q"], d["kv"], st.idx, wl.scale, st.out, st.lse, None, st.ws)
+
+    ms_f, clk = time_calls(fused_step, steps, warmup, flush)
+    same = bool(torch.equal(st.idx, dsa_idx))
+    ms_s, _ = time_calls(st.run, steps, warmup, flush)
+    out["decode_128k_fused_topk"] = {
+        "what": "decode step with the fused indexer -> top-k call vs the separate calls (same selection)",
+        "fused_ms_per_step": round(ms_f, 4), "separate_ms_per_step": round(ms_s, 4),
+        "same_selection": same, "clocks": clk}
     block, r = 64, 64
     sums = torch.empty(B, L // block, wl.d_I, device=device)
     dsa.dsa_hisa_block_sums(d["kI"], block, sums)  # cache summary: once, outside the timed steps

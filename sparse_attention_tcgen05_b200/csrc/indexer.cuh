@@ -179,48 +179,68 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
+    // The whole warp walks the items; lane 0 waits and issues the copies.  Decode: the rows of
+    // the next 16 tiles' 64-key boxes are looked up together, one per lane (a paged cache reads
+    // its block table: 32 loads in flight instead of one at a time in the issuing thread).
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
-      const uint64_t evict_first = l2_evict_first_policy();
-      int ks = 0;
-      uint32_t kph = 0;
-      int qi = 0;
-      for (int u = blockIdx.x; u < p.n_items; u += gridDim.x) {
-        int b, qg, kc, kt0, kt1, n_comp;
-        decode_item(p, u, b, qg, kc);
-        item_tiles<G>(p, b, qg, kc, kt0, kt1, n_comp);
-        if (n_comp == 0) continue;
-        const int qb = qi & 1;
-        const uint32_t qph = (qi >> 1) & 1;
-        if (!mbar_wait(&q_empty[qb], qph ^ 1, abort_flag, 1)) goto done;
-        mbar_arrive_expect_tx(&q_full[qb], C::kQBytes);
-        tma_load_2d(sQ + qb * ((C::kQBytes + 1023) / 1024) * 1024, &tm_q, &q_full[qb], 0,
-                    (b * p.Lq + qg * G) * H_I);
-        for (int tt = 0; tt < n_comp; ++tt) {
-          if (!mbar_wait(&k_empty[ks], kph ^ 1, abort_flag, 2)) goto done;
-          mbar_arrive_expect_tx(&k_full[ks], C::kKBytes);
-          if constexpr (G == 1) {
-            // two boxes of 64 keys; a box past the query (or the sequence) is read as zeros from
-            // one row past the tensor, never through the page table
-            const int t_row = query_pos(p, b, qg);
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const int s0 = (kt0 + tt) * kTileKeys + h * C::kKBox;
-              const long y = s0 <= t_row ? key_row(p, b, s0) : -1;
-              tma_load_2d_hint(sK + ks * C::kKBytes + h * C::kKBox * D_I, &tm_k, &k_full[ks], 0,
-                               y >= 0 ? static_cast<int32_t>(y) : p.k_rows, evict_first);
-            }
-          } else {
-            tma_load_2d(sK + ks * C::kKBytes, &tm_k, &k_full[ks], 0, b * p.Lk + (kt0 + tt) * kTileKeys);
-          }
-          if (++ks == C::kStages) {
-            ks = 0;
-            kph ^= 1;
+    }
+    const uint64_t evict_first = l2_evict_first_policy();
+    int ks = 0;
+    uint32_t kph = 0;
+    int qi = 0;
+    for (int u = blockIdx.x; u < p.n_items; u += gridDim.x) {
+      int b, qg, kc, kt0, kt1, n_comp;
+      decode_item(p, u, b, qg, kc);
+      item_tiles<G>(p, b, qg, kc, kt0, kt1, n_comp);
+      if (n_comp == 0) continue;
+      const int qb = qi & 1;
+      const uint32_t qph = (qi >> 1) & 1;
+      bool got = true;
+      if (lane == 0) {
+        got = mbar_wait(&q_empty[qb], qph ^ 1, abort_flag, 1);
+        if (got) {
+          mbar_arrive_expect_tx(&q_full[qb], C::kQBytes);
+          tma_load_2d(sQ + qb * ((C::kQBytes + 1023) / 1024) * 1024, &tm_q, &q_full[qb], 0,
+                      (b * p.Lq + qg * G) * H_I);
+        }
+      }
+      if (!__all_sync(0xFFFFFFFFu, got)) goto done;
+      const int t_row = (G == 1) ? query_pos(p, b, qg) : 0;  // decode: the query's position
+      long my_row = -1;                                      // decode: box `lane` of the window
+      for (int tt = 0; tt < n_comp; ++tt) {
+        if constexpr (G == 1) {
+          if ((tt & 15) == 0) {
+            // a box past the query (or the sequence) is read as zeros from one row past the
+            // tensor, never through the page table
+            const int s0 = (kt0 + tt + (lane >> 1)) * kTileKeys + (lane & 1) * C::kKBox;
+            my_row = (tt + (lane >> 1) < n_comp && s0 <= t_row) ? key_row(p, b, s0) : -1;
           }
         }
-        ++qi;
+        const long y0 = __shfl_sync(0xFFFFFFFFu, my_row, 2 * (tt & 15));
+        const long y1 = __shfl_sync(0xFFFFFFFFu, my_row, 2 * (tt & 15) + 1);
+        if (lane == 0) {
+          got = mbar_wait(&k_empty[ks], kph ^ 1, abort_flag, 2);
+          if (got) {
+            mbar_arrive_expect_tx(&k_full[ks], C::kKBytes);
+            if constexpr (G == 1) {
+              tma_load_2d_hint(sK + ks * C::kKBytes, &tm_k, &k_full[ks], 0,
+                               y0 >= 0 ? static_cast<int32_t>(y0) : p.k_rows, evict_first);
+              tma_load_2d_hint(sK + ks * C::kKBytes + C::kKBox * D_I, &tm_k, &k_full[ks], 0,
+                               y1 >= 0 ? static_cast<int32_t>(y1) : p.k_rows, evict_first);
+            } else {
+              tma_load_2d(sK + ks * C::kKBytes, &tm_k, &k_full[ks], 0, b * p.Lk + (kt0 + tt) * kTileKeys);
+            }
+          }
+        }
+        if (!__all_sync(0xFFFFFFFFu, got)) goto done;
+        if (++ks == C::kStages) {
+          ks = 0;
+          kph ^= 1;
+        }
       }
+      ++qi;
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
@@ -284,6 +304,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       decode_item(p, u, b, qg, kc);
       item_tiles<G>(p, b, qg, kc, kt0, kt1, n_comp);
       const int i0 = qg * G;
+      int t_item = 0;  // decode: the query's position, read once per item
+      if constexpr (G == 1) t_item = query_pos(p, b, i0);
       float* wbuf = sW + (it & 1) * C::N;
       for (int x = e; x < C::N; x += 256) {
         const int i = i0 + x / H_I;
@@ -325,19 +347,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int g = 0; g < C::kQPerWG; ++g) {
             const int i = i0 + wg * C::kQPerWG * (C::kSplitWG ? 1 : 0) + g;
             if (i < p.Lq) {
-              const int t = query_pos(p, b, i);
+              const int t = (G == 1) ? t_item : query_pos(p, b, i);
               p.scores[(row_base + i) * p.Lk + s] = (s <= t) ? acc[g] : -INFINITY;
             }
           }
         }
         if constexpr (G == 1) {
           if (count) {
-            // the tile's visible scores by top digit: one shared atomic per distinct digit and
-            // warp (integer-valued scores crowd into a few digits)
-            const int t = query_pos(p, b, i0);
-            const uint32_t bin = (s < p.Lk && s <= t) ? (ordered_key(acc[0]) >> 21) : 0xFFFFFFFFu;
-            const uint32_t peers = __match_any_sync(0xFFFFFFFFu, bin);
-            if (bin != 0xFFFFFFFFu && lane == __ffs(peers) - 1) atomicAdd(&gHist[bin], __popc(peers));
+            // the tile's visible scores by top digit (plain shared atomics: aggregating equal
+            // digits over the warp first measured slower)
+            if (s < p.Lk && s <= t_item) atomicAdd(&gHist[ordered_key(acc[0]) >> 21], 1u);
           }
         }
       }

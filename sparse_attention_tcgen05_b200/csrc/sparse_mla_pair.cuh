@@ -308,7 +308,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t dst_off = bx < 4 ? static_cast<uint32_t>(bx * kMainBox + g * 512) : static_cast<uint32_t>(4 * kMainBox + g * 256);
     const int npairs = (total + 1) / 2;
     auto slot_of = [&](int j) { return j < total ? block_slot(p, idx_row, e0, len, j < nblk ? j : j - nblk, lane) : -1; };
-    int next_lo = (total > 0) ? slot_of(0) : -1, next_hi = (total > 1) ? slot_of(1) : -1;
+    // two-deep pipeline of the lookups: the slots (idx loads) two pairs ahead, the rows (a block
+    // table load for a paged cache) one pair ahead
+    auto row_of = [&](int sv) {
+      if (sv >= len_b) record_bad_index();
+      return mla::kv_row(p, b, len_b, sv);
+    };
+    int y_nlo = row_of((total > 0) ? slot_of(0) : -1), y_nhi = row_of((total > 1) ? slot_of(1) : -1);
+    int s_nlo = slot_of(2), s_nhi = slot_of(3);
     int issued = 0;
     if (lane == 0) {
       tma_prefetch_desc(&tm_main);
@@ -320,14 +327,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool got = jp != 1 || mbar_wait(q_ready, 0, abort_flag, 66);
       got = got && mbar_wait(&kv_empty[st], ((jp / kStages) & 1) ^ 1, abort_flag, 62);
       if (!__all_sync(0xFFFFFFFFu, got)) break;  // the shuffles below need the whole warp
-      const int s_lo = next_lo, s_hi = next_hi;
+      const int y_lo = y_nlo, y_hi = y_nhi;
       if (jp + 1 < npairs) {
-        next_lo = slot_of(2 * jp + 2);
-        next_hi = slot_of(2 * jp + 3);
+        y_nlo = row_of(s_nlo);
+        y_nhi = row_of(s_nhi);
+        s_nlo = slot_of(2 * jp + 4);
+        s_nhi = slot_of(2 * jp + 5);
       }
-      if (s_lo >= len_b || s_hi >= len_b) record_bad_index();
-      const int y_lo = mla::kv_row(p, b, len_b, s_lo);
-      const int y_hi = mla::kv_row(p, b, len_b, s_hi);
       const int src = 4 * (g & 7);
       int yv[4];
 #pragma unroll
