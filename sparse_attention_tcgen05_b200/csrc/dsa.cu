@@ -199,7 +199,7 @@ dsa_status launch_indexer(const void* q, const void* kk, const float* w, float* 
       cudaSuccess)
     return DSA_ERR_CUDA;
   const int grid = static_cast<int>(std::min<long>(items, sms));
-  return launch(kern, static_cast<unsigned>(grid), dsa::indexer::kThreads, Cfg::kSmemBytes, stream, 1, tm_q, tm_k, p);
+  return launch(kern, static_cast<unsigned>(grid), Cfg::kThreads, Cfg::kSmemBytes, stream, 1, tm_q, tm_k, p);
 }
 
 // ------------------------------------------------------------------------------ top-k

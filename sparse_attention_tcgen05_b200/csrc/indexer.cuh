@@ -14,7 +14,8 @@
 //                 there for the top-k.
 //   warp 1        MMA issuer (one thread): d_I/32 MMAs of 128 x N x 32 per tile
 //   warp 2        TMEM allocator (2 accumulators of N columns, double-buffered)
-//   warps 4..11   epilogue: tcgen05.ld -> ReLU * w -> head sum -> mask -> store; for decode
+//   warps 4..     epilogue, 2 or 4 warpgroups: tcgen05.ld -> ReLU * w -> head sum -> mask ->
+//                 store; for decode
 //                 with a `hist` buffer (the fused indexer -> top-k path) it also counts every
 //                 visible score of the row by the top 11 bits of its order-preserving key, the
 //                 top-k's first radix digit (shared-memory counts per work item, added to the
@@ -30,8 +31,6 @@
 namespace dsa {
 namespace indexer {
 
-constexpr int kEpiWarps = 8;
-constexpr int kThreads = 128 + kEpiWarps * 32;
 constexpr int kTileKeys = 128;
 
 struct Params {
@@ -64,10 +63,15 @@ struct Cfg {
   static constexpr int kKBytes = kTileKeys * D_I;        // k_I tile
   static constexpr int kTmemCols = (2 * N <= 32) ? 32 : (2 * N <= 64) ? 64 : (2 * N <= 128) ? 128
                                    : (2 * N <= 256) ? 256 : 512;
-  static constexpr bool kSplitWG = (G >= 2);             // two epilogue warpgroups split queries
-  static constexpr int kColsPerWG = kSplitWG ? N / 2 : N;
-  static constexpr int kQPerWG = kSplitWG ? G / 2 : 1;
-  static constexpr int kEpiWorkers = kSplitWG ? 256 : 128;
+  // Epilogue warpgroups: four for prefill with at least 32 heads (the ReLU-weighted head sum is
+  // the kernel's ALU load, spread over 16 warps), two otherwise.
+  static constexpr int kEpiGroups = (G >= 4 && H_I >= 32) ? 4 : 2;
+  static constexpr int kEpiThreads = kEpiGroups * 128;
+  static constexpr int kThreads = 128 + kEpiThreads;
+  static constexpr bool kSplitWG = (G >= 2);             // the epilogue warpgroups split queries
+  static constexpr int kColsPerWG = kSplitWG ? N / kEpiGroups : N;
+  static constexpr int kQPerWG = kSplitWG ? G / kEpiGroups : 1;
+  static constexpr int kEpiWorkers = kSplitWG ? kEpiThreads : 128;
   static constexpr uint32_t kSwizzle = D_I == 128 ? kSw128 : D_I == 64 ? kSw64 : kSw32;
   static constexpr uint32_t kIdesc = make_idesc(0, 0, false, false, 128, N);
   // shared memory layout (offsets from a 1024-aligned base)
@@ -130,7 +134,7 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
 }
 
 template <int H_I, int D_I, int G>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Cfg<H_I, D_I, G>::kThreads, 1)
     indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const Params p) {
   using C = Cfg<H_I, D_I, G>;
@@ -286,8 +290,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------------ epilogue
-    const int e = threadIdx.x - 128;  // 0..255
-    const int wg = e >> 7;            // warpgroup 0 / 1
+    const int e = threadIdx.x - 128;  // 0 .. kEpiThreads - 1
+    const int wg = e >> 7;            // epilogue warpgroup
     const int sp = warp & 3;          // TMEM sub-partition this warp may access
     const int row = sp * 32 + lane;   // accumulator row = key within the tile
     // G >= 2: both groups take every tile (half of the queries each).  G == 1: the groups take
@@ -307,11 +311,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       int t_item = 0;  // decode: the query's position, read once per item
       if constexpr (G == 1) t_item = query_pos(p, b, i0);
       float* wbuf = sW + (it & 1) * C::N;
-      for (int x = e; x < C::N; x += 256) {
+      for (int x = e; x < C::N; x += C::kEpiThreads) {
         const int i = i0 + x / H_I;
         wbuf[x] = (i < p.Lq) ? p.w[(static_cast<size_t>(b) * p.Lq + i) * H_I + (x % H_I)] : 0.f;
       }
-      named_bar_sync(1, 256);
+      named_bar_sync(1, C::kEpiThreads);
       const size_t row_base = static_cast<size_t>(b) * p.Lq;
       for (int tt = 0; tt < n_comp; ++tt, ++gt) {
         const int ab = gt & 1;
@@ -374,7 +378,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // fully masked tiles: no MMA, just -inf
       for (int kt = kt0 + n_comp; ok && kt < kt1; ++kt) {
-        for (int x = e; x < G * kTileKeys; x += 256) {
+        for (int x = e; x < G * kTileKeys; x += C::kEpiThreads) {
           const int i = i0 + x / kTileKeys;
           const int s = kt * kTileKeys + (x % kTileKeys);
           if (i < p.Lq && s < p.Lk) p.scores[(row_base + i) * p.Lk + s] = -INFINITY;
