@@ -6,7 +6,7 @@ batch of seeded synthetic inputs, plus each stage's roofline fraction.
                   [--scaling weak|strong] [--no-extra] [--peaks] [--dry-run]
 
 Default workload: long_prefill_32k (B=1, L=32768 causal, the largest single-GPU workload). With
-N = 1 the same JSON line also carries a benchmark spec block (the 128K-context decode, B=32 queries
+N = 1 the same JSON line also carries a `decode_128k` block (the 128K-context decode, B=32 queries
 against 131072 keys each) and a `workloads` block with every other workload, each timed the same
 way with fewer steps.
 
@@ -49,7 +49,7 @@ from sparse_attention_tcgen05_b200.sharding import (MLA_WEIGHT, max_over_ranks, 
 
 METRIC = "query-tokens/s (indexer+top-k+sparse MLA) at 1 B200; % of roofline per stage"
 DEFAULT_WORKLOAD = "long_prefill_32k"
-NORTH_STAR = "decode_128k"
+DECODE_TARGET = "decode_128k"  # the decode workload held to a path-roofline target
 L2_FLUSH_BYTES = 512 << 20
 # FP8 e4m3 dense rate relative to bf16 (NVIDIA B200 datasheet, dense: 4.5 vs 2.25 PFLOP/s)
 FP8_OVER_BF16 = 2.0
@@ -717,7 +717,7 @@ def gpu_arm(args, rank, world, device):
     if world == 1 and not args.no_extra:
         # every other workload, timed the same way (fewer steps, no host round trip)
         extra = {}
-        names = [NORTH_STAR] + [n for n in ("decode_32k", "prefill_2x8k", "indexer_kl_16k", "dense_warmup_16k",
+        names = [DECODE_TARGET] + [n for n in ("decode_32k", "prefill_2x8k", "indexer_kl_16k", "dense_warmup_16k",
                                             "tiny_prefill") if n != args.workload]
         for name in names:
             if name == args.workload:
@@ -729,12 +729,12 @@ def gpu_arm(args, rank, world, device):
             r.pop("e2e")
             r["config"] = workload_config(w2)
             extra[name] = r
-        if NORTH_STAR in extra:
-            line["north_star"] = extra.pop(NORTH_STAR)
-            line["north_star"]["target"] = "path_roofline_frac >= 0.60"
+        if DECODE_TARGET in extra:
+            line[DECODE_TARGET] = extra.pop(DECODE_TARGET)
+            line[DECODE_TARGET]["target"] = "path_roofline_frac >= 0.60"
         line["workloads"] = extra
         line["gpu_launches"] += sum(r["gpu_launches"] for r in extra.values()) + \
-            line.get("north_star", {}).get("gpu_launches", 0)
+            line.get(DECODE_TARGET, {}).get("gpu_launches", 0)
         torch.cuda.empty_cache()
         line["variants"] = variant_blocks(device, peaks, args.extra_steps, 3)
     return line

@@ -122,6 +122,24 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// The same wait, polling without suspending: for chains of short waits (the sparse attention's
+// softmax and gather roles), where the thread's wake-up after a suspension costs more than the
+// issue slots the polling takes from the other warps (measured: the attention 1.6 % faster, the
+// decode indexer's producer 8 % slower with it, so it is not the default).
+__device__ __forceinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parity, volatile int* abort, int site) {
+  if (mbar_test_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+    if (mbar_test_wait(bar, parity)) return true;
+    if (*abort) return false;
+    if (global_timer_ns() - t0 > wait_limit_ns()) {
+      record_timeout(site);
+      *abort = 1;
+      return false;
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------------------------
 // Thread-block clusters: distributed shared memory and cross-CTA mbarrier arrivals
 // ---------------------------------------------------------------------------------------------

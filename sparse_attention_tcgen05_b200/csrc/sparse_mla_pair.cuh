@@ -241,7 +241,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kMmaWarp) {
     // ------------------------------------------------------------------ MMA issuer (polling)
     if (lane == 0 && total > 0) {
-      if (!mbar_wait(q_ready, 0, abort_flag, 60)) goto done;
+      if (!mbar_wait_spin(q_ready, 0, abort_flag, 60)) goto done;
       tc_fence_after();
       const uint32_t q_tmem = tmem_base + kTmemQ;
       const int npairs = (total + 1) / 2;
@@ -324,8 +324,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int jp = 0; jp < npairs; ++jp) {
       const int st = jp % kStages;
       // stages 1.. hold the staged Q until it is in tensor memory
-      bool got = jp != 1 || mbar_wait(q_ready, 0, abort_flag, 66);
-      got = got && mbar_wait(&kv_empty[st], ((jp / kStages) & 1) ^ 1, abort_flag, 62);
+      bool got = jp != 1 || mbar_wait_spin(q_ready, 0, abort_flag, 66);
+      got = got && mbar_wait_spin(&kv_empty[st], ((jp / kStages) & 1) ^ 1, abort_flag, 62);
       if (!__all_sync(0xFFFFFFFFu, got)) break;  // the shuffles below need the whole warp
       const int y_lo = y_nlo, y_hi = y_nhi;
       if (jp + 1 < npairs) {
@@ -381,7 +381,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // from the TMA-staged slice (row h of a box; 16-byte chunk c sits at c ^ (h & 7) in a
     // 128-byte row, at c ^ ((h >> 1) & 3) in a 64-byte rope row).  Heads >= H get zeros.  The
     // staged slice is waited for even with no work, so no copy is in flight at exit.
-    if (!mbar_wait(q_full, 0, abort_flag, 65)) {
+    if (!mbar_wait_spin(q_full, 0, abort_flag, 65)) {
       ok = false;
       if (threadIdx.x == 0) mbar_drain(q_full, 0);  // let the staged copy land before exit
     }
@@ -430,7 +430,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (wtid == 0) bulk_wait_read_all();
       named_bar_sync(bar_xs, 128);
       uint32_t v[32];
-      if (ok && !mbar_wait(&s_full[0], (q >> 1) & 1, abort_flag, 63)) ok = false;
+      if (ok && !mbar_wait_spin(&s_full[0], (q >> 1) & 1, abort_flag, 63)) ok = false;
       ok = __all_sync(0xFFFFFFFFu, ok);  // tcgen05.ld is warp-collective
       if (ok) {
         tc_fence_after();
@@ -503,7 +503,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (nblk == 0) return;
       const int ql = nblk - 1;
       if (ok) {
-        const bool got = mbar_wait(&o_done[ql & 1], (ql >> 1) & 1, abort_flag, 67);
+        const bool got = mbar_wait_spin(&o_done[ql & 1], (ql >> 1) & 1, abort_flag, 67);
         ok = __all_sync(0xFFFFFFFFu, got);
       }
       if (!ok) return;
@@ -591,7 +591,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                fmaxf(fmaxf(m8[2], m8[6]), fmaxf(m8[3], m8[7]))) * sc;
         float rp = -INFINITY;
         if (q > 0) {
-          if (ok && !mbar_wait(&ref_full[(q - 1) & 1], ((q - 1) >> 1) & 1, abort_flag, 68)) ok = false;
+          if (ok && !mbar_wait_spin(&ref_full[(q - 1) & 1], ((q - 1) >> 1) & 1, abort_flag, 68)) ok = false;
           ok = __all_sync(0xFFFFFFFFu, ok);
           rp = sRef[((q - 1) & 1) * 128 + h];
         }
@@ -601,12 +601,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ---- step 4: rescale O if the reference moved, then P
         const int pb = q & 1;
         if (ok && q >= 2) {  // P buffer pb was last read by PV(q-2)
-          const bool got = mbar_wait(&o_done[pb], ((q - 2) >> 1) & 1, abort_flag, 65);
+          const bool got = mbar_wait_spin(&o_done[pb], ((q - 2) >> 1) & 1, abort_flag, 65);
           ok = __all_sync(0xFFFFFFFFu, got);
         }
         const bool moved = (rp != -INFINITY) && (rq != rp);
         if (ok && __any_sync(0xFFFFFFFFu, moved)) {
-          const bool got = mbar_wait(&o_done[(q - 1) & 1], ((q - 1) >> 1) & 1, abort_flag, 66);
+          const bool got = mbar_wait_spin(&o_done[(q - 1) & 1], ((q - 1) >> 1) & 1, abort_flag, 66);
           ok = __all_sync(0xFFFFFFFFu, got);
           if (ok) {
             const float f = moved ? ex2_approx(rp - rq) : 1.f;
