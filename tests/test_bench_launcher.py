@@ -83,3 +83,36 @@ def test_a_causal_shard_reproduces_the_whole_sequence_rows():
         np.testing.assert_array_equal(part["scores"], whole["scores"][rows, :loc.Lk])
         np.testing.assert_allclose(part["out"], whole["out"][rows], rtol=0, atol=0)
         np.testing.assert_allclose(part["kl"], whole["kl"][rows], rtol=0, atol=0)
+
+
+def test_algorithmic_work_and_roofline_by_hand():
+    # the per-stage byte and MAC counts the roofline fractions divide by, recomputed by hand for
+    # the 128K decode rows and a causal prefill, and the bound each stage takes
+    bench = _bench()
+    wl = dsa_inputs.WORKLOADS["decode_128k"]
+    w = bench.algorithmic(wl)
+    B, L, k = 32, 131072, 2048
+    assert w["indexer"]["bytes"] == B * L * 128 + B * 64 * (128 + 4) + B * L * 4
+    assert w["indexer"]["macs"] == B * L * 64 * 128
+    assert w["topk"]["bytes"] == 4 * B * L + 4 * B * k
+    assert w["sparse_mla"]["macs"] == B * k * 128 * (576 + 512)
+    # q + idx + the selected latents (k distinct rows per sequence) + out + lse
+    assert w["sparse_mla"]["bytes"] == 2 * B * 128 * 576 + 4 * B * k + 2 * B * k * 576 + 2 * B * 128 * 512 + 4 * B * 128
+    peaks = {"hbm_gbs": 6550.1, "bf16_tflops": 1660.8, "bf16_tflops_sustained": 1384.5}
+    us, bound = bench.roofline_us("indexer", w["indexer"], peaks)
+    assert bound == "hbm" and abs(us - w["indexer"]["bytes"] / 6550.1e3) < 1e-6
+    us, bound = bench.roofline_us("sparse_mla", w["sparse_mla"], peaks)
+    tc = 2 * w["sparse_mla"]["macs"] / 1660.8e6
+    assert bound == ("tensor" if tc > w["sparse_mla"]["bytes"] / 6550.1e3 else "hbm")
+    # causal prefill: pairs and selected entries summed over t = 0 .. L-1
+    wl = dsa_inputs.WORKLOADS["prefill_2x8k"]
+    w = bench.algorithmic(wl)
+    L = 8192
+    pairs = 2 * L * (L + 1) // 2
+    nsel = 2 * sum(min(k, t + 1) for t in range(L))
+    assert w["indexer"]["macs"] == pairs * 64 * 128
+    assert w["sparse_mla"]["macs"] == nsel * 128 * 1088
+    us, bound = bench.roofline_us("sparse_mla", w["sparse_mla"], peaks)
+    assert bound == "tensor" and abs(us - 2 * nsel * 128 * 1088 / 1660.8e6) < 1e-6
+    us, bound = bench.roofline_us("indexer", w["indexer"], peaks)  # FP8 at twice the bf16 figure
+    assert bound == "tensor" and abs(us - 2 * pairs * 64 * 128 / (2 * 1660.8e6)) < 1e-6
