@@ -48,6 +48,39 @@ def test_indexer_bit_exact(dsa, H_I, d_I, B, Lq, Lk):
         np.testing.assert_array_equal(got[b, i], exp, err_msg=f"row {r}")
 
 
+def test_indexer_large_batch_decode_walks_whole_rows(dsa):
+    # with at least two rows per SM a work item is a whole sequence (33 key tiles here), so the
+    # producer refills its 16-tile window of box rows mid-item; contiguous rows against the oracle
+    # (sampled), and a shuffled paged copy of the same cache against the contiguous call
+    B, Lk, H_I, d_I, k, P = 300, 4224, 64, 128, 256, 64
+    wl = dsa_inputs.custom("ix_wide_batch", 4242, B, 1, Lk, H_I, d_I, 16, k, 1, 16, 16)
+    dw = parity.DeviceWorkload(wl, with_attention=False)
+    scores = torch.full((B, 1, Lk), float("nan"), dtype=torch.float32, device="cuda")
+    dsa.dsa_indexer(dw.qI, dw.kI, dw.w, scores)
+    got = scores.cpu().numpy()
+    assert dsa.dsa_last_device_status() == 0
+    qI = dw.qI_np.reshape(B, H_I, d_I)
+    w = dw.w_np.reshape(B, H_I)
+    for b in (0, 1, 77, 148, 149, 150, 222, 296, 297, 299):
+        exp = ref.indexer_row(qI[b], dw.kI_np[b], w[b], Lk - 1).astype(np.float32)
+        np.testing.assert_array_equal(got[b, 0], exp, err_msg=f"row {b}")
+    # the same cache as pages of 64 keys in a shuffled pool, every row full
+    pages = Lk // P
+    g = torch.Generator().manual_seed(99)
+    table = torch.randperm(B * pages, generator=g).to(torch.int32).reshape(B, pages).cuda()
+    pool = torch.empty(B * pages, P, d_I, dtype=dw.kI.dtype, device="cuda")
+    pool.view(torch.uint8)[table.flatten().long()] = dw.kI.reshape(B * pages, P, d_I).view(torch.uint8)
+    lens = torch.full((B,), Lk, dtype=torch.int32, device="cuda")
+    s1, s2 = (torch.empty(B, 1, Lk, device="cuda") for _ in range(2))
+    i1, i2 = (torch.empty(B, 1, k, dtype=torch.int32, device="cuda") for _ in range(2))
+    ws_ix = torch.zeros(dsa.dsa_workspace_bytes(dsa.DSA_OP_INDEXER_TOPK, B, 1, Lk, k, 0), dtype=torch.uint8,
+                        device="cuda")
+    dsa.dsa_indexer_topk_paged(dw.qI, pool, dw.w, table, lens, s1, i1, ws_ix)
+    dsa.dsa_indexer_topk(dw.qI, dw.kI, dw.w, s2, i2, ws_ix)
+    assert dsa.dsa_last_device_status() == 0
+    assert torch.equal(s1, scores) and torch.equal(s2, scores) and torch.equal(i1, i2)
+
+
 def test_indexer_rejects_bad_arguments(dsa):
     q = torch.zeros(1, 4, 64, 128, dtype=torch.float8_e4m3fn, device="cuda")
     k = torch.zeros(1, 8, 128, dtype=torch.float8_e4m3fn, device="cuda")
