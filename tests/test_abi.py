@@ -56,6 +56,44 @@ def test_host_validation_rejects_without_touching_a_device(lib):
     assert lib.dsa_indexer_kl_noalloc(fake, fake, fake, 1, 4, 8, 4, fake, odd, None) == 1
 
 
+
+def test_host_validation_of_the_variant_entry_points(lib):
+    # bad arguments and unsupported shapes of the dense, backward, paged, HISA and masked-MHA calls
+    # answer before any device work (1 = DSA_ERR_INVALID_ARG, 2 = DSA_ERR_UNSUPPORTED)
+    P = ctypes.c_void_p
+    fake, odd = P(0x10000), P(0x10004)
+    nan = float("nan")
+    # dense warm-up: null output, Lq > Lk, non-finite scale, more than 128 heads
+    assert lib.dsa_dense_mla_fwd(fake, fake, 1, 8, 8, 128, 576, 512, 0.1, None, None, None, None, 0, None) == 1
+    assert lib.dsa_dense_mla_fwd(fake, fake, 1, 9, 8, 128, 576, 512, 0.1, fake, None, None, None, 0, None) == 1
+    assert lib.dsa_dense_mla_fwd(fake, fake, 1, 8, 8, 128, 576, 512, nan, fake, None, None, None, 0, None) == 1
+    assert lib.dsa_dense_mla_fwd(fake, fake, 1, 8, 8, 129, 576, 512, 0.1, fake, None, None, None, 0, None) == 2
+    # dense KL: no per-row output and no workspace; misaligned per-row output
+    assert lib.dsa_indexer_kl_dense(fake, fake, 1, 8, 8, fake, None, None, 0, None) == 1
+    assert lib.dsa_indexer_kl_dense(fake, fake, 1, 8, 8, fake, odd, None, 0, None) == 1
+    # backward: a dense call (idx = NULL) must take every position; other head shapes
+    assert lib.dsa_indexer_bwd(fake, fake, fake, fake, None, fake, 1, 4, 8, 64, 128, 4, fake, fake, fake, None) == 1
+    assert lib.dsa_indexer_bwd(fake, fake, fake, fake, fake, fake, 1, 4, 8, 32, 128, 4, fake, fake, fake, None) == 2
+    # paged decode: pages must hold a multiple of 64 entries; the table must be given
+    assert lib.dsa_indexer_topk_paged(fake, fake, fake, fake, fake, fake, fake, 2, 4096, 100, 48, 64, 128, 256,
+                                      fake, 1 << 20, None) == 2
+    assert lib.dsa_indexer_topk_paged(fake, fake, fake, None, fake, fake, fake, 2, 4096, 100, 64, 64, 128, 256,
+                                      fake, 1 << 20, None) == 1
+    assert lib.dsa_sparse_mla_fwd_paged(fake, fake, fake, fake, fake, 2, 4096, 100, 64, 128, 576, 256, 256, 0.1,
+                                        fake, None, fake, 1 << 20, None) == 2
+    # HISA: whole blocks of a multiple of 64 keys; d_I = 128 for the block sums
+    assert lib.dsa_hisa_block_sums(fake, 2, 4096, 64, 64, fake, None) == 2
+    assert lib.dsa_hisa_topk(fake, fake, fake, fake, 2, 4096, 64, 128, 96, 8, 256, fake, None, fake, 1 << 20,
+                             None) == 2
+    assert lib.dsa_hisa_topk(fake, fake, fake, fake, 2, 4096, 64, 128, 64, 8, 256, fake, None, None, 0,
+                             None) == 1
+    # masked MHA: 192/128-dim heads only; the workspace is required
+    assert lib.dsa_masked_mha_fwd(fake, fake, fake, fake, 1, 256, 8, 128, 128, 32, 0.1, fake, None, fake,
+                                  1 << 20, None) == 2
+    assert lib.dsa_masked_mha_fwd(fake, fake, fake, fake, 1, 256, 8, 192, 128, 32, 0.1, fake, None, None, 0,
+                                  None) == 1
+
+
 def test_workspace_sizes(lib):
     import sparse_attention_tcgen05_b200 as dsa
     assert dsa.dsa_workspace_bytes(dsa.DSA_OP_INDEXER, 1, 1, 8, 4, 8) == 0
